@@ -1,0 +1,387 @@
+"""Benchmark of the CSA2 decode step over an FP4 global KV cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference]
+                    [--config 3]
+
+One step = one decode step of a whole CSA2 layer group (csa2_layer_group):
+Full-layer indexer scan + HSI pool + Top-512, Reindex rescoring, Reuse, and
+sparse + SWA attention of every layer.  The default workload is the 1M-context
+20-layer decoder stack (batch 1, context 1,048,576, [F,R,R,R] + 4 x [X,R,R,R],
+64 planted blocks).  Metric: decode layer-steps/s (batch x layers / step time).
+
+Timing: CUDA events on the launching stream around every step, L2 flushed
+(256 MiB write) between steps outside the events, W warm-up steps, max over
+ranks.  --gpus N > 1 runs N independent replicas (the decode step has no
+exchange to make across GPUs), one per rank, launched by torchrun.
+The reference arm (--impl reference) times the CPU oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s and achieved HBM GB/s vs 8 TB/s at 128K–1M ctx"
+UNIT = "layer-steps/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+ATTN_BYTES = 512 * 288 + 128 * 512 + 2 * 16384 + 2048   # per layer per sequence
+
+
+def algorithmic_bytes(wl) -> dict:
+    """Bytes the method must move per step (intermediates excluded)."""
+    C = wl.n_rows.astype(np.int64)
+    full = int(sum(128 * int(c) for c in C)) * int((wl.modes == 0).sum())
+    pool_pos = min(wl.pool_blocks, 1 << 30) * 8 if wl.pool_blocks else None
+    rx = 0
+    for _ in range(int((wl.modes == 1).sum())):
+        rx += int(sum(128 * (min(pool_pos, int(c)) if pool_pos else int(c)) for c in C))
+    attn = ATTN_BYTES * wl.B * wl.L
+    return {"scan": full, "reindex": rx, "attn": attn, "total": full + rx + attn}
+
+
+def measured_peaks() -> tuple[float, str]:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def scan_traffic_from_profile():
+    """dram bytes per scan launch from the committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", "scan_decoder20_1m.md")
+    try:
+        with open(path) as fh:
+            for line in fh:
+                if line.startswith("dram_bytes_per_launch:"):
+                    return int(line.split(":", 1)[1].strip().split()[0])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """NVML sampling of SM clock and throttle reasons while running."""
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ ranks
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The largest x over all ranks (device time of the slowest replica)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, t_ms: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest time."""
+    return units_per_rank * world / (t_ms * 1e-3)
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def oracle_step_time(wl, budget_s: float = 30.0):
+    """Time the CPU oracle's layer group on this workload: one full step.
+
+    The oracle reads main-KV codes only at the rows it selects, so a first
+    (untimed) pass with zero codes finds those rows, the oracle quantises them
+    from the seeded bf16 rows, and the timed pass runs on the real bytes."""
+    import oracle
+
+    dm = oracle.dims()
+    x_sel_rows = None
+    rows_needed = set()
+    codes = np.zeros((wl.pool_rows, 256), np.uint8)
+    scales = np.zeros((wl.pool_rows, 32), np.uint8)
+    idxk = np.zeros((wl.pool_rows, 64), np.uint16)
+    for r0, _, kc in wl.iter_chunks():
+        idxk[r0:r0 + len(kc)] = kc
+    kv = oracle.KV(codes, scales, idxk, seq_stride=wl.seq_stride, page_table=wl.page_table)
+    r = oracle.layer_group(kv, dm, wl.n_rows, wl.modes, wl.q_idx, wl.w_h, wl.q, wl.swa,
+                           wl.swa_len, top_k=wl.top_k, pool_blocks=wl.pool_blocks)
+    for l in range(wl.L):
+        for b in range(wl.B):
+            pos = r["idx"][l, b, :r["idx_count"][l, b]]
+            rows_needed.update(wl.row_of(b, pos).tolist())
+    x_sel_rows = np.array(sorted(rows_needed), dtype=np.int64)
+    xs, _ = wl.rows(x_sel_rows)
+    c, s = oracle.quantize_fp4(xs)
+    kv.codes[x_sel_rows] = c
+    kv.scales[x_sel_rows] = s
+    t0 = time.perf_counter()
+    oracle.layer_group(kv, dm, wl.n_rows, wl.modes, wl.q_idx, wl.w_h, wl.q, wl.swa, wl.swa_len,
+                       top_k=wl.top_k, pool_blocks=wl.pool_blocks)
+    dt = time.perf_counter() - t0
+    return dt
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    dt = oracle_step_time(wl)
+    value = wl.B * wl.L / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": 1, "warmup": 0, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(wl),
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": 1,
+                             "sample": f"one full decode step of {wl.name} (single-threaded C, "
+                                       "fp64, full-sort selection)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl):
+    return {"workload": wl.name, "batch": int(wl.B), "context": int(wl.n_rows.max()),
+            "layers": int(wl.L), "modes": "".join("FXR"[m] for m in wl.modes),
+            "top_k": int(wl.top_k), "pool_blocks": int(wl.pool_blocks),
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+# ------------------------------------------------------------ GPU arm
+def run_gpu(args, wl, rank, world):
+    import torch
+
+    from fp4_kv_cache_quantize_b200 import csa2
+
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_
+        import datetime
+        dist_.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_
+
+    def barrier():
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(dev)
+
+    # ---- setup: FP4 cache via the library's pack kernel, indexer K, inputs
+    rows = wl.pool_rows
+    codes = torch.empty((rows, 256), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, 32), dtype=torch.uint8, device=dev)
+    idxk = torch.empty((rows, 64), dtype=torch.int16, device=dev)
+    for r0, xc, kc in wl.iter_chunks():
+        n = len(xc)
+        csa2.csa2_quantize_fp4(to_dev(xc).view(torch.bfloat16), codes[r0:r0 + n],
+                               scales[r0:r0 + n])
+        idxk[r0:r0 + n] = to_dev(kc)
+    n_rows = to_dev(wl.n_rows.astype(np.int32))
+    pt = None if wl.page_table is None else to_dev(wl.page_table)
+    kv = csa2.KVCache(codes, scales, idxk, n_rows, max_rows=int(wl.n_rows.max()),
+                      seq_stride=wl.seq_stride, page_table=pt)
+    q_idx, w_h, q = to_dev(wl.q_idx), to_dev(wl.w_h), to_dev(wl.q)
+    swa, swa_len = to_dev(wl.swa), to_dev(wl.swa_len)
+    grp = csa2.LayerGroup(kv, wl.modes, q_idx, w_h, q, swa, swa_len, top_k=wl.top_k,
+                          pool_blocks=wl.pool_blocks)
+    ws = csa2.workspace(grp.workspace_size(), device=dev)
+    csa2.csa2_workspace_init(ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa2.csa2_layer_group(grp, ws)
+
+    for _ in range(args.warmup):
+        step()
+    csa2.csa2_sync_status(ws)
+
+    # ---- timed device loop
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    sampler = ClockSampler(local)
+    barrier()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    csa2.csa2_sync_status(ws)
+    times = [a.elapsed_time(b) for a, b in ev]   # ms
+    t_step = max_over_ranks(sum(times) / K, dist, dev)
+
+    # ---- traced pass: per-launch events for the stage breakdown and roofline
+    n_ev = 16
+    tev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev * K)]
+    for e in tev:
+        e.record(stream)
+    torch.cuda.synchronize()
+    traces = []
+    for i in range(K):
+        tr = csa2.Trace(tev[i * n_ev:(i + 1) * n_ev])
+        flush.zero_()
+        csa2.csa2_trace_set(tr)
+        step()
+        csa2.csa2_trace_set(None)
+        traces.append(tr)
+    torch.cuda.synchronize()
+    stage_tot, stage_n, launches = {}, {}, 0
+    for tr in traces:
+        names = tr.names()
+        launches = len(names) - 1
+        for j in range(len(names) - 1):
+            d = tr.events[j].elapsed_time(tr.events[j + 1])
+            stage_tot[names[j]] = stage_tot.get(names[j], 0.0) + d
+            stage_n[names[j]] = stage_n.get(names[j], 0) + 1
+    stage_us_step = {k: 1e3 * v / K for k, v in stage_tot.items()}       # per step
+    stage_us_launch = {k: 1e3 * v / stage_n[k] for k, v in stage_tot.items()}  # per launch
+
+    # ---- end to end through the C ABI with host buffers
+    h_q_idx = torch.from_numpy(np.ascontiguousarray(wl.q_idx).view(np.int16)).pin_memory()
+    h_w = torch.from_numpy(np.ascontiguousarray(wl.w_h)).pin_memory()
+    h_q = torch.from_numpy(np.ascontiguousarray(wl.q).view(np.int16)).pin_memory()
+    h_out = torch.empty(grp.out.shape, dtype=torch.bfloat16).pin_memory()
+    h_idx = torch.empty(grp.idx.shape, dtype=torch.int32).pin_memory()
+    h2d = h_q_idx.numel() * 2 + h_w.numel() * 4 + h_q.numel() * 2
+    d2h = h_out.numel() * 2 + h_idx.numel() * 4
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(K)]
+    barrier()
+    for i in range(K):
+        flush.zero_()
+        e_ev[i][0].record(stream)
+        q_idx.copy_(h_q_idx, non_blocking=True)
+        w_h.copy_(h_w, non_blocking=True)
+        q.copy_(h_q, non_blocking=True)
+        step()
+        h_out.copy_(grp.out, non_blocking=True)
+        h_idx.copy_(grp.idx, non_blocking=True)
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / K, dist, dev)
+
+    units = wl.B * wl.L
+    value = job_throughput(units, world, t_step)
+    ab = algorithmic_bytes(wl)
+    peak, peak_kind = measured_peaks()
+    scan_us = stage_us_launch.get("scan")
+    roof = None
+    if scan_us:
+        achieved = ab["scan"] / max(1, int((wl.modes == 0).sum())) / (scan_us * 1e-6) / 1e9
+        roof = {"bound": "hbm", "kernel": "score_scan_kernel", "achieved": achieved,
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": achieved / peak, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                "traffic": scan_traffic_from_profile(),
+                "algorithmic_bytes_per_launch": ab["scan"] // max(1, int((wl.modes == 0).sum()))}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        dt = oracle_step_time(wl)
+        cpu = {"value": units / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"one full decode step of {wl.name} on one host core (fp64 C oracle)"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(wl),
+            "hbm_gbs_algorithmic": ab["total"] / (t_step * 1e-3) / 1e9,
+            "algorithmic_bytes_per_step": ab["total"],
+            "stage_us": stage_us_step,
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": job_throughput(units, world, t_e2e), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": int(launches * K),
+            "gpu_launches_per_step": int(launches),
+            "clocks": sampler.summary(),
+            "step_ms_p10_p50_p90": [float(np.percentile(times, p)) for p in (10, 50, 90)]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    from fp4_kv_cache_quantize_b200 import synth
+    wl = synth.config(args.config)
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+    run_gpu(args, wl, rank, world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,455 @@
+// capi_index.cu -- C ABI of the indexer, the attention and the layer group:
+// host-side checks, workspace layout, TMA tensor maps, and the launch DAG.
+//
+// Layer group schedule (release note section "Compressed Sparse Attention 2
+// (CSA2)"; yomxxx.com CSA2 notes, section 二, mode table and HSI paragraph):
+//   for each FULL layer f:
+//     scan(q_f) -> block maxima -> block Top-P (P = pool_blocks, or top_k
+//     blocks when there is no pool) -> rescore + Top-k of f and of every
+//     REINDEX layer up to the next FULL layer (one launch; they depend only
+//     on the pool) ;
+//   REINDEX without a pool: its own scan -> block Top-k -> rescore + Top-k ;
+//   one attention launch for every layer (REUSE layers read the indices of
+//   the latest FULL/REINDEX layer) ; one merge launch when split-KV is used.
+// Exact Top-k of a FULL layer over all positions is taken over the positions
+// of its Top-P blocks: every one of the k best positions lies in a block whose
+// maximum is among the k best block maxima (ties to the lower position and
+// block), so P >= k blocks hold them all.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <vector>
+
+#include "capi_common.h"
+#include "csa2_internal.cuh"
+#include "kernels.h"
+
+namespace csa2 {
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over rows of 64 values (128 B), 128B swizzle, zero OOB fill.
+static csa2_status map_rows64(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t gdim[2] = {64, rows < 1 ? 1 : rows};
+  cuuint64_t gstride[1] = {128};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return CSA2_OK;
+}
+
+// ------------------------------------------------------------ validation
+static csa2_status check_kv(const csa2_kv_view* kv) {
+  CSA2_REQUIRE(kv != nullptr, CSA2_ERR_INVALID_ARG, "kv is NULL");
+  CSA2_REQUIRE_PTR(kv->codes);
+  CSA2_REQUIRE_PTR(kv->scales);
+  CSA2_REQUIRE_PTR(kv->idx_k);
+  CSA2_REQUIRE(kv->n_rows != nullptr, CSA2_ERR_INVALID_ARG, "kv->n_rows is NULL");
+  CSA2_REQUIRE(kv->batch >= 1 && kv->batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", kv->batch);
+  CSA2_REQUIRE(kv->max_rows >= 0 && kv->max_rows <= CSA2_MAX_ROWS, CSA2_ERR_SHAPE,
+               "max_rows = %d outside [0, %d]", kv->max_rows, (int)CSA2_MAX_ROWS);
+  CSA2_REQUIRE(kv->pool_rows >= 0 && kv->pool_rows <= (int64_t)0x7FFF0000, CSA2_ERR_SHAPE,
+               "pool_rows = %lld", (long long)kv->pool_rows);
+  if (kv->page_table) {
+    CSA2_REQUIRE(kv->page_rows == 64, CSA2_ERR_SHAPE, "page_rows = %d (must be 64)", kv->page_rows);
+    CSA2_REQUIRE((int64_t)kv->max_pages * 64 >= kv->max_rows, CSA2_ERR_SHAPE,
+                 "max_pages = %d cannot hold max_rows = %d", kv->max_pages, kv->max_rows);
+  } else {
+    CSA2_REQUIRE(kv->seq_stride >= kv->max_rows, CSA2_ERR_SHAPE,
+                 "seq_stride = %lld < max_rows = %d", (long long)kv->seq_stride, kv->max_rows);
+    CSA2_REQUIRE(kv->seq_stride % 64 == 0, CSA2_ERR_ALIGNMENT,
+                 "seq_stride = %lld is not a multiple of 64 rows", (long long)kv->seq_stride);
+    CSA2_REQUIRE((int64_t)(kv->batch - 1) * kv->seq_stride + kv->max_rows <= kv->pool_rows,
+                 CSA2_ERR_SHAPE, "the row pool of %lld rows is too small for the layout",
+                 (long long)kv->pool_rows);
+  }
+  return CSA2_OK;
+}
+
+static csa2_status check_topk(int top_k, int pool_blocks) {
+  CSA2_REQUIRE(top_k >= 1 && top_k <= CSA2_MAX_TOPK, CSA2_ERR_SHAPE, "top_k = %d outside [1, %d]",
+               top_k, (int)CSA2_MAX_TOPK);
+  CSA2_REQUIRE(pool_blocks == 0 || (pool_blocks >= top_k && pool_blocks <= CSA2_MAX_POOL),
+               CSA2_ERR_SHAPE, "pool_blocks = %d must be 0 or in [top_k, %d]", pool_blocks,
+               (int)CSA2_MAX_POOL);
+  return CSA2_OK;
+}
+
+// ------------------------------------------------------------ workspace
+struct IndexWs {
+  uint32_t* status;
+  float* bm;
+  int32_t bm_stride;
+  int32_t* sel;
+  int32_t* sel_count;
+  int32_t sel_stride;
+  size_t bytes;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static IndexWs index_ws_layout(const csa2_kv_view* kv, int top_k, uint8_t* base) {
+  IndexWs w{};
+  const int nblk = (kv->max_rows + CSA2_BLK - 1) / CSA2_BLK;
+  w.bm_stride = ((nblk + 15) / 16) * 16;
+  if (w.bm_stride == 0) w.bm_stride = 16;
+  w.sel_stride = top_k;
+  size_t off = CSA2_WS_HEADER;
+  w.status = reinterpret_cast<uint32_t*>(base);
+  w.bm = reinterpret_cast<float*>(base + off);
+  off = align256(off + (size_t)kv->batch * w.bm_stride * sizeof(float));
+  w.sel = reinterpret_cast<int32_t*>(base + off);
+  off = align256(off + (size_t)kv->batch * w.sel_stride * sizeof(int32_t));
+  w.sel_count = reinterpret_cast<int32_t*>(base + off);
+  off = align256(off + (size_t)kv->batch * sizeof(int32_t));
+  w.bytes = off;
+  return w;
+}
+
+static ScanParams scan_params(const csa2_kv_view* kv, const float* w, const IndexWs& ws) {
+  ScanParams p{};
+  p.n_rows = kv->n_rows;
+  p.page_table = kv->page_table;
+  p.max_pages = kv->max_pages;
+  p.max_rows = kv->max_rows;
+  p.seq_stride = kv->seq_stride;
+  p.pool_rows = kv->pool_rows;
+  p.w = w;
+  p.bm = ws.bm;
+  p.bm_stride = ws.bm_stride;
+  p.batch = kv->batch;
+  p.tiles_per_seq = (kv->max_rows + SC_TILE - 1) / SC_TILE;
+  p.status = ws.status;
+  return p;
+}
+
+static RescoreParams rescore_params(const csa2_kv_view* kv, const int32_t* cand,
+                                    const int32_t* cand_count, int cand_stride, int top_k,
+                                    uint32_t* status) {
+  RescoreParams p{};
+  p.idx_k = kv->idx_k;
+  p.page_table = kv->page_table;
+  p.max_pages = kv->max_pages;
+  p.max_rows = kv->max_rows;
+  p.seq_stride = kv->seq_stride;
+  p.pool_rows = kv->pool_rows;
+  p.n_rows = kv->n_rows;
+  p.cand = cand;
+  p.cand_count = cand_count;
+  p.cand_stride = cand_stride;
+  p.top_k = top_k;
+  p.status = status;
+  return p;
+}
+
+// scan + block select: candidates (top P blocks by block max) into sel
+static csa2_status run_scan_select(const csa2_kv_view* kv, const uint16_t* q_idx, const float* w,
+                                   int P, int32_t* sel, int32_t* sel_count, int sel_stride,
+                                   const IndexWs& ws, cudaStream_t st) {
+  CUtensorMap map_k, map_q;
+  csa2_status r = map_rows64(&map_k, kv->idx_k, (uint64_t)kv->pool_rows, 64);
+  if (r) return r;
+  r = map_rows64(&map_q, q_idx, (uint64_t)kv->batch * CSA2_HI, 16);
+  if (r) return r;
+  trace_mark("scan", st);
+  CSA2_CUDA(launch_scan(map_k, map_q, scan_params(kv, w, ws), num_sms(), st));
+  trace_mark("block_select", st);
+  CSA2_CUDA(launch_block_select(ws.bm, ws.bm_stride, kv->n_rows, kv->max_rows, kv->batch, P, sel,
+                                sel_stride, sel_count, ws.status, st));
+  return CSA2_OK;
+}
+
+static int cand_blocks_max(const csa2_kv_view* kv, int P) {
+  const int nblk = (kv->max_rows + CSA2_BLK - 1) / CSA2_BLK;
+  return P < nblk ? P : nblk;
+}
+
+// ------------------------------------------------------------ group plan
+struct GroupWs {
+  IndexWs ix;
+  float* part_o;
+  float* part_ml;
+  int nsplit;
+  size_t bytes;
+};
+
+static GroupWs group_ws_layout(const csa2_group_desc* d, uint8_t* base) {
+  GroupWs g{};
+  g.ix = index_ws_layout(&d->kv, d->top_k, base);
+  g.nsplit = attn_nsplit(d->kv.batch * d->n_layers, num_sms());
+  size_t off = g.ix.bytes;
+  const size_t pb = attn_partial_bytes(d->kv.batch, d->n_layers, g.nsplit);
+  const size_t pairs = (size_t)d->kv.batch * d->n_layers * g.nsplit;
+  g.part_o = reinterpret_cast<float*>(base + off);
+  g.part_ml = reinterpret_cast<float*>(base + off + pairs * CSA2_H * CSA2_D * sizeof(float));
+  off = align256(off + pb);
+  g.bytes = off;
+  return g;
+}
+
+}  // namespace csa2
+
+using namespace csa2;
+
+extern "C" {
+
+size_t csa2_index_workspace_size(const csa2_kv_view* kv, int32_t top_k, int32_t pool_blocks) {
+  (void)pool_blocks;
+  if (!kv || top_k < 1) return 0;
+  return index_ws_layout(kv, top_k, nullptr).bytes;
+}
+
+csa2_status csa2_index_full(const csa2_kv_view* kv, const uint16_t* q_idx, const float* w,
+                            int32_t top_k, int32_t pool_blocks, int32_t* idx, int32_t* idx_count,
+                            int32_t* pool, int32_t* pool_count, void* ws, size_t ws_bytes,
+                            csa2_stream_t stream) {
+  csa2_status r = check_kv(kv);
+  if (r) return r;
+  if ((r = check_topk(top_k, pool_blocks))) return r;
+  CSA2_REQUIRE_PTR(q_idx);
+  CSA2_REQUIRE_PTR(w);
+  CSA2_REQUIRE_PTR(idx);
+  CSA2_REQUIRE_PTR(idx_count);
+  CSA2_REQUIRE_PTR(ws);
+  if (pool_blocks > 0) {
+    CSA2_REQUIRE_PTR(pool);
+    CSA2_REQUIRE_PTR(pool_count);
+  }
+  const IndexWs lay = index_ws_layout(kv, top_k, static_cast<uint8_t*>(ws));
+  CSA2_REQUIRE(ws_bytes >= lay.bytes, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
+               lay.bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int P = pool_blocks > 0 ? pool_blocks : top_k;
+  int32_t* sel = pool_blocks > 0 ? pool : lay.sel;
+  int32_t* sel_count = pool_blocks > 0 ? pool_count : lay.sel_count;
+  const int sel_stride = pool_blocks > 0 ? pool_blocks : lay.sel_stride;
+  if ((r = run_scan_select(kv, q_idx, w, P, sel, sel_count, sel_stride, lay, st))) return r;
+  RescoreParams rp = rescore_params(kv, sel, sel_count, sel_stride, top_k, lay.status);
+  rp.job[0] = RescoreJob{q_idx, w, idx, idx_count, top_k};
+  trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, 1, kv->batch, cand_blocks_max(kv, P), st));
+  trace_mark("end", st);
+  return CSA2_OK;
+}
+
+csa2_status csa2_index_reindex(const csa2_kv_view* kv, const uint16_t* q_idx, const float* w,
+                               const int32_t* pool, const int32_t* pool_count,
+                               int32_t pool_stride, int32_t top_k, int32_t* idx,
+                               int32_t* idx_count, void* ws, size_t ws_bytes,
+                               csa2_stream_t stream) {
+  csa2_status r = check_kv(kv);
+  if (r) return r;
+  if ((r = check_topk(top_k, 0))) return r;
+  CSA2_REQUIRE_PTR(q_idx);
+  CSA2_REQUIRE_PTR(w);
+  CSA2_REQUIRE_PTR(idx);
+  CSA2_REQUIRE_PTR(idx_count);
+  CSA2_REQUIRE_PTR(ws);
+  const IndexWs lay = index_ws_layout(kv, top_k, static_cast<uint8_t*>(ws));
+  CSA2_REQUIRE(ws_bytes >= lay.bytes, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
+               lay.bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (pool) {
+    CSA2_REQUIRE_PTR(pool_count);
+    CSA2_REQUIRE(pool_stride >= 1 && pool_stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
+                 "pool_stride = %d outside [1, %d]", pool_stride, (int)CSA2_MAX_POOL);
+    RescoreParams rp = rescore_params(kv, pool, pool_count, pool_stride, top_k, lay.status);
+    rp.job[0] = RescoreJob{q_idx, w, idx, idx_count, top_k};
+    trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, 1, kv->batch, cand_blocks_max(kv, pool_stride), st));
+    trace_mark("end", st);
+    return CSA2_OK;
+  }
+  if ((r = run_scan_select(kv, q_idx, w, top_k, lay.sel, lay.sel_count, lay.sel_stride, lay, st)))
+    return r;
+  RescoreParams rp = rescore_params(kv, lay.sel, lay.sel_count, lay.sel_stride, top_k, lay.status);
+  rp.job[0] = RescoreJob{q_idx, w, idx, idx_count, top_k};
+  trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, 1, kv->batch, cand_blocks_max(kv, top_k), st));
+  trace_mark("end", st);
+  return CSA2_OK;
+}
+
+size_t csa2_attn_workspace_size(int32_t batch, int32_t n_layers) {
+  if (batch < 1 || n_layers < 1) return 0;
+  const int ns = attn_nsplit(batch * n_layers, num_sms());
+  return CSA2_WS_HEADER + align256(attn_partial_bytes(batch, n_layers, ns));
+}
+
+static csa2_status fill_attn_common(AttnParams& ap, const csa2_kv_view* kv, const int32_t* swa_len,
+                                    float sm_scale, int idx_stride) {
+  ap.batch = kv->batch;
+  ap.idx_stride = idx_stride;
+  ap.codes = kv->codes;
+  ap.scales = kv->scales;
+  ap.page_table = kv->page_table;
+  ap.max_pages = kv->max_pages;
+  ap.max_rows = kv->max_rows;
+  ap.seq_stride = kv->seq_stride;
+  ap.pool_rows = kv->pool_rows;
+  ap.n_rows = kv->n_rows;
+  ap.swa_len = swa_len;
+  ap.scale_log2 = sm_scale * 1.4426950408889634f;
+  return CSA2_OK;
+}
+
+csa2_status csa2_sparse_attn_decode(const uint16_t* q, const csa2_kv_view* kv, const int32_t* idx,
+                                    const int32_t* idx_count, int32_t idx_stride,
+                                    const uint8_t* swa, const int32_t* swa_len, float sm_scale,
+                                    uint16_t* out, void* ws, size_t ws_bytes,
+                                    csa2_stream_t stream) {
+  csa2_status r = check_kv(kv);
+  if (r) return r;
+  CSA2_REQUIRE_PTR(q);
+  CSA2_REQUIRE_PTR(idx);
+  CSA2_REQUIRE_PTR(idx_count);
+  CSA2_REQUIRE_PTR(swa);
+  CSA2_REQUIRE_PTR(swa_len);
+  CSA2_REQUIRE_PTR(out);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(idx_stride >= 1 && idx_stride <= CSA2_MAX_TOPK, CSA2_ERR_SHAPE,
+               "idx_stride = %d outside [1, %d]", idx_stride, (int)CSA2_MAX_TOPK);
+  CSA2_REQUIRE(sm_scale == sm_scale, CSA2_ERR_INVALID_ARG, "sm_scale is NaN");
+  const size_t need = csa2_attn_workspace_size(kv->batch, 1);
+  CSA2_REQUIRE(ws_bytes >= need, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  AttnParams ap{};
+  fill_attn_common(ap, kv, swa_len, sm_scale, idx_stride);
+  ap.n_layers = 1;
+  ap.nsplit = attn_nsplit(kv->batch, num_sms());
+  ap.layer[0] = AttnLayer{q, swa, idx, idx_count, nullptr, nullptr, out};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t pairs = (size_t)kv->batch * ap.nsplit;
+  ap.part_o = reinterpret_cast<float*>(base + CSA2_WS_HEADER);
+  ap.part_ml = reinterpret_cast<float*>(base + CSA2_WS_HEADER + pairs * CSA2_H * CSA2_D * 4);
+  ap.status = reinterpret_cast<uint32_t*>(base);
+  CSA2_CUDA(launch_attn(ap, (cudaStream_t)stream));
+  trace_mark("end", (cudaStream_t)stream);
+  return CSA2_OK;
+}
+
+size_t csa2_group_workspace_size(const csa2_group_desc* d) {
+  if (!d || d->n_layers < 1 || d->top_k < 1 || d->kv.batch < 1) return 0;
+  return group_ws_layout(d, nullptr).bytes;
+}
+
+csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes,
+                             csa2_stream_t stream) {
+  CSA2_REQUIRE(d != nullptr, CSA2_ERR_INVALID_ARG, "desc is NULL");
+  const csa2_kv_view* kv = &d->kv;
+  csa2_status r = check_kv(kv);
+  if (r) return r;
+  if ((r = check_topk(d->top_k, d->pool_blocks))) return r;
+  const int L = d->n_layers, B = kv->batch;
+  CSA2_REQUIRE(L >= 1 && L <= AT_MAX_LAYERS, CSA2_ERR_SHAPE, "n_layers = %d outside [1, %d]", L,
+               AT_MAX_LAYERS);
+  CSA2_REQUIRE(d->modes != nullptr, CSA2_ERR_INVALID_ARG, "modes is NULL");
+  for (int l = 0; l < L; l++)
+    CSA2_REQUIRE(d->modes[l] >= CSA2_FULL && d->modes[l] <= CSA2_REUSE, CSA2_ERR_INVALID_ARG,
+                 "modes[%d] = %d", l, d->modes[l]);
+  CSA2_REQUIRE(d->modes[0] == CSA2_FULL, CSA2_ERR_INVALID_ARG,
+               "layer 0 must be FULL (REINDEX and REUSE reuse an earlier FULL layer's cache)");
+  CSA2_REQUIRE_PTR(d->q_idx);
+  CSA2_REQUIRE_PTR(d->w);
+  CSA2_REQUIRE_PTR(d->q);
+  CSA2_REQUIRE_PTR(d->swa);
+  CSA2_REQUIRE_PTR(d->swa_len);
+  CSA2_REQUIRE_PTR(d->idx);
+  CSA2_REQUIRE_PTR(d->idx_count);
+  CSA2_REQUIRE_PTR(d->out);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(d->sm_scale == d->sm_scale, CSA2_ERR_INVALID_ARG, "sm_scale is NaN");
+  if (d->pool_blocks > 0) {
+    CSA2_REQUIRE_PTR(d->pool);
+    CSA2_REQUIRE_PTR(d->pool_count);
+  }
+  const GroupWs g = group_ws_layout(d, static_cast<uint8_t*>(ws));
+  CSA2_REQUIRE(ws_bytes >= g.bytes, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes,
+               g.bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int K = d->top_k;
+  const size_t qi_stride = (size_t)B * CSA2_HI * CSA2_DI, w_stride = (size_t)B * CSA2_HI;
+  auto layer_idx = [&](int l) { return d->idx + (size_t)l * B * K; };
+  auto layer_cnt = [&](int l) { return d->idx_count + (size_t)l * B; };
+
+  // Indexer: per FULL layer, one scan + block select and one rescore launch
+  // for the FULL layer and the REINDEX layers that share its pool.
+  const bool hsi = d->pool_blocks > 0;
+  for (int l = 0; l < L; l++) {
+    if (d->modes[l] == CSA2_REUSE) continue;
+    if (d->modes[l] == CSA2_REINDEX && hsi) continue;  // batched with its FULL layer
+    const uint16_t* qi = d->q_idx + l * qi_stride;
+    const float* wl = d->w + l * w_stride;
+    const int P = hsi ? d->pool_blocks : K;
+    int32_t* sel = hsi ? d->pool : g.ix.sel;
+    int32_t* sel_count = hsi ? d->pool_count : g.ix.sel_count;
+    const int sel_stride = hsi ? d->pool_blocks : g.ix.sel_stride;
+    if ((r = run_scan_select(kv, qi, wl, P, sel, sel_count, sel_stride, g.ix, st))) return r;
+    RescoreParams rp = rescore_params(kv, sel, sel_count, sel_stride, K, g.ix.status);
+    int nj = 0;
+    rp.job[nj++] = RescoreJob{qi, wl, layer_idx(l), layer_cnt(l), K};
+    if (hsi && d->modes[l] == CSA2_FULL) {
+      for (int x = l + 1; x < L && d->modes[x] != CSA2_FULL; x++) {
+        if (d->modes[x] != CSA2_REINDEX) continue;
+        if (nj == RS_MAX_JOBS) {
+          trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, nj, B, cand_blocks_max(kv, P), st));
+          nj = 0;
+        }
+        rp.job[nj++] =
+            RescoreJob{d->q_idx + x * qi_stride, d->w + x * w_stride, layer_idx(x), layer_cnt(x), K};
+      }
+    }
+    trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, nj, B, cand_blocks_max(kv, P), st));
+  }
+
+  // Attention for every layer in one launch.
+  AttnParams ap{};
+  fill_attn_common(ap, kv, d->swa_len, d->sm_scale, K);
+  ap.n_layers = L;
+  ap.nsplit = g.nsplit;
+  ap.part_o = g.part_o;
+  ap.part_ml = g.part_ml;
+  ap.status = g.ix.status;
+  int src = 0;
+  for (int l = 0; l < L; l++) {
+    if (d->modes[l] != CSA2_REUSE) src = l;
+    const bool reuse = d->modes[l] == CSA2_REUSE;
+    ap.layer[l] = AttnLayer{d->q + (size_t)l * B * CSA2_H * CSA2_D,
+                            d->swa + (size_t)l * B * CSA2_W * CSA2_D,
+                            layer_idx(src),
+                            layer_cnt(src),
+                            reuse ? layer_idx(l) : nullptr,
+                            reuse ? layer_cnt(l) : nullptr,
+                            d->out + (size_t)l * B * CSA2_H * CSA2_D};
+  }
+  CSA2_CUDA(launch_attn(ap, st));
+  trace_mark("end", st);
+  return CSA2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// kernels.h -- launch interfaces between the C ABI (capi*.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+void trace_mark(const char* stage, cudaStream_t st);  // capi.cu
+
+// score.cu -------------------------------------------------------------
+struct ScanParams {
+  const int32_t* n_rows;
+  const int32_t* page_table;
+  int32_t max_pages;
+  int32_t max_rows;
+  int64_t seq_stride;
+  int64_t pool_rows;
+  const float* w;
+  float* bm;
+  int32_t bm_stride;
+  int32_t batch;
+  int32_t tiles_per_seq;
+  uint32_t* status;
+};
+constexpr int SC_TILE = 128;
+
+constexpr int RS_MAX_JOBS = 8;
+struct RescoreJob {
+  const uint16_t* q_idx;
+  const float* w;
+  int32_t* idx;
+  int32_t* idx_count;
+  int32_t idx_stride;
+};
+struct RescoreParams {
+  RescoreJob job[RS_MAX_JOBS];
+  const uint16_t* idx_k;
+  const int32_t* page_table;
+  int32_t max_pages;
+  int32_t max_rows;
+  int64_t seq_stride;
+  int64_t pool_rows;
+  const int32_t* n_rows;
+  const int32_t* cand;
+  const int32_t* cand_count;
+  int32_t cand_stride;
+  int32_t top_k;
+  uint32_t* status;
+};
+
+cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
+                        int num_sms, cudaStream_t st);
+cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
+                           cudaStream_t st);
+cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n_rows,
+                                int max_rows, int batch, int k_req, int32_t* sel, int sel_stride,
+                                int32_t* sel_count, uint32_t* status, cudaStream_t st);
+
+// attn.cu --------------------------------------------------------------
+constexpr int AT_MAX_LAYERS = 32;
+struct AttnLayer {
+  const uint16_t* q;
+  const uint8_t* swa;
+  const int32_t* idx;
+  const int32_t* idx_count;
+  int32_t* idx_copy;
+  int32_t* idx_copy_count;
+  uint16_t* out;
+};
+struct AttnParams {
+  AttnLayer layer[AT_MAX_LAYERS];
+  int32_t n_layers, batch, idx_stride, nsplit;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const int32_t* page_table;
+  int32_t max_pages;
+  int32_t max_rows;
+  int64_t seq_stride;
+  int64_t pool_rows;
+  const int32_t* n_rows;
+  const int32_t* swa_len;
+  float scale_log2;
+  float* part_o;
+  float* part_ml;
+  uint32_t* status;
+};
+int attn_nsplit(int pairs, int num_sms);
+size_t attn_partial_bytes(int batch, int n_layers, int nsplit);
+cudaError_t launch_attn(const AttnParams& p, cudaStream_t st);
+
+}  // namespace csa2

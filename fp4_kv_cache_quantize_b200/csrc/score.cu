@@ -1,0 +1,478 @@
+// score.cu -- the CSA2 indexer kernels.
+//
+//  * score_scan_kernel: the Full-mode scan [release note, section
+//    "Compressed Sparse Attention 2 (CSA2)": the Full layer scores every
+//    causally visible position; yomxxx.com CSA2 notes, section 二, HSI
+//    paragraph: it keeps the top 2,048 blocks of 8 positions by block max].
+//    It streams the bf16 indexer K (128 B per position) from HBM with TMA
+//    into a 5-stage shared-memory ring (128B-swizzled tiles of 128 positions),
+//    one thread issues tcgen05.mma (M = 128 positions, N = 16 >= 8 indexer
+//    heads, K = 64) into a double-buffered TMEM accumulator, and four
+//    epilogue warps read the dot products back (tcgen05.ld), apply
+//    s = sum_h w_h * relu(q_h . k), and write only the block maxima of
+//    8-position blocks.  Scores themselves never touch HBM.
+//  * rescore_select_kernel: scores the positions of a set of candidate blocks
+//    (the HSI pool for Reindex layers, the Full layer's top blocks for its own
+//    Top-512) with legacy mma.sync tensor-core tiles over gathered rows, then
+//    selects the exact Top-k in the same cluster with the radix select of
+//    select.cuh.  Several (layer, sequence) jobs run in one launch.
+#include <cuda_bf16.h>
+
+#include "csa2_internal.cuh"
+#include "kernels.h"
+#include "select.cuh"
+
+namespace csa2 {
+
+// ------------------------------------------------------------- the scan
+constexpr int SC_BOX = 64;                 // rows per TMA box
+constexpr int SC_N = 16;                   // indexer heads padded to MMA N
+constexpr int SC_STAGES = 5;
+constexpr int SC_A_BYTES = SC_TILE * 128;  // 16 KB of indexer K per stage
+constexpr int SC_B_BYTES = SC_N * 128;     // 2 KB of indexer query per stage
+constexpr int SC_THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr uint32_t SC_IDESC = idesc_bf16_f32(SC_TILE, SC_N);
+
+struct ScanSmem {
+  uint8_t a[SC_STAGES][SC_A_BYTES];
+  uint8_t b[SC_STAGES][SC_B_BYTES];
+  uint64_t full[SC_STAGES], empty[SC_STAGES];
+  uint64_t tfull[2], tempty[2], done;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t SC_SMEM = sizeof(ScanSmem) + 1024;
+
+
+__device__ __forceinline__ int visible_rows(const int32_t* n_rows, int b, int max_rows,
+                                            uint32_t* status) {
+  int c = n_rows[b];
+  if (c < 0 || c > max_rows) {
+    set_status(status, ST_DEVICE_CHECK);
+    c = c < 0 ? 0 : max_rows;
+  }
+  return c;
+}
+
+// First pool row of the 64-row box holding position pos0 (a multiple of 64),
+// or pool_rows (out of range: TMA fills zeros) when the row map is invalid.
+__device__ __forceinline__ int32_t box_row(const ScanParams& p, int b, int pos0) {
+  int64_t row;
+  if (p.page_table) {
+    const int page = pos0 / SC_BOX;
+    const int64_t pid = page < p.max_pages ? (int64_t)p.page_table[(int64_t)b * p.max_pages + page]
+                                           : -1;
+    row = pid * SC_BOX;
+    if (pid < 0 || row + SC_BOX > p.pool_rows) {
+      set_status(p.status, ST_DEVICE_CHECK);
+      row = p.pool_rows;
+    }
+  } else {
+    row = (int64_t)b * p.seq_stride + pos0;
+  }
+  return (int32_t)row;
+}
+
+__global__ void __launch_bounds__(SC_THREADS, 1)
+    score_scan_kernel(const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_q, const ScanParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  ScanSmem& s = *reinterpret_cast<ScanSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id(), lane = lane_id();
+  const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SC_STAGES; i++) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 4 * 32);
+    }
+    mbar_init(&s.done, 1);
+    s.abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_q);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 32);  // two 16-column fp32 accumulators
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abort = &s.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_phase = 0;
+      for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+        const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
+        const int C = visible_rows(p.n_rows, b, p.max_rows, p.status);
+        if (t * SC_TILE >= C) continue;
+        if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort)) {
+          s.abort = 1;
+          set_status(p.status, ST_TIMEOUT);
+          break;
+        }
+        const int pos0 = t * SC_TILE;
+        const int32_t y0 = box_row(p, b, pos0);
+        const int32_t y1 = pos0 + SC_BOX < C ? box_row(p, b, pos0 + SC_BOX) : y0;
+        mbar_arrive_expect_tx(&s.full[stage], SC_A_BYTES + SC_B_BYTES);
+        tma_load_2d(s.a[stage], &map_k, &s.full[stage], 0, y0);
+        tma_load_2d(s.a[stage] + SC_BOX * 128, &map_k, &s.full[stage], 0, y1);
+        tma_load_2d(s.b[stage], &map_q, &s.full[stage], 0, b * CSA2_HI);
+        issued |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == SC_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      // Drain: every issued copy lands before the CTA may exit.
+      for (int i = 0; i < SC_STAGES; i++)
+        if ((issued >> i) & 1u)
+          if (!mbar_wait(&s.full[i], (issued_phase >> i) & 1u, nullptr))
+            set_status(p.status, ST_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------------------------- MMA issuer
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+        const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
+        const int C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
+        if (t * SC_TILE >= C) continue;
+        if (!mbar_wait(&s.full[stage], phase, abort) ||
+            !mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort)) {
+          s.abort = 1;
+          set_status(p.status, ST_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(s.a[stage]), b_addr = smem_u32(s.b[stage]);
+        const uint32_t d = tmem + (uint32_t)(acc * SC_N);
+#pragma unroll
+        for (int k = 0; k < 4; k++)  // K = 64 as four K = 16 steps inside the swizzle atom
+          umma_bf16(d, sdesc_k128(a_addr + 32 * k), sdesc_k128(b_addr + 32 * k), SC_IDESC,
+                    k > 0);
+        umma_commit(&s.empty[stage]);
+        umma_commit(&s.tfull[acc]);
+        if (++stage == SC_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      umma_commit(&s.done);  // completes once every MMA issued above has
+      if (!mbar_wait(&s.done, 0, nullptr)) set_status(p.status, ST_TIMEOUT);
+    }
+  } else {  // ------------------------------------------ epilogue, 4 warps
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int cur_b = -1;
+    float w[CSA2_HI];
+    for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+      const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
+      const int C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
+      if (t * SC_TILE >= C) continue;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.tfull[acc], acc_phase, abort));
+      if (!ok) {
+        s.abort = 1;
+        set_status(p.status, ST_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[8];
+      tmem_ld_x8(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * SC_N), r);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s.tempty[acc]);
+      if (b != cur_b) {
+#pragma unroll
+        for (int h = 0; h < CSA2_HI; h++) w[h] = __ldg(p.w + b * CSA2_HI + h);
+        cur_b = b;
+      }
+      float sc = 0.0f;
+#pragma unroll
+      for (int h = 0; h < CSA2_HI; h++) sc = fmaf(w[h], fmaxf(__uint_as_float(r[h]), 0.0f), sc);
+      const int pos = t * SC_TILE + row;
+      if (pos >= C) sc = -INFINITY;
+      sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
+      sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
+      sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
+      if ((lane & 7) == 0 && pos < C) p.bm[(int64_t)b * p.bm_stride + pos / CSA2_BLK] = sc;
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
+// ------------------------------------------------- rescore + Top-k select
+constexpr int RS_NT = 256;
+
+
+
+template <int KPT>
+struct RescoreSmem {
+  SelectSmem<RS_NT> sel;
+  uint32_t keys[RS_NT * KPT];
+  int32_t blocks[RS_NT * KPT / CSA2_BLK];
+};
+
+__device__ __forceinline__ int64_t pos_row(const RescoreParams& p, int b, int pos) {
+  if (p.page_table) {
+    const int page = pos >> 6;
+    const int64_t pid =
+        page < p.max_pages ? (int64_t)p.page_table[(int64_t)b * p.max_pages + page] : -1;
+    const int64_t row = pid * 64 + (pos & 63);
+    return (pid < 0 || row >= p.pool_rows) ? -1 : row;
+  }
+  const int64_t row = (int64_t)b * p.seq_stride + pos;
+  return row < p.pool_rows ? row : -1;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int KPT>
+__global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescoreParams p) {
+  constexpr int EPC = RS_NT * KPT;  // candidates per CTA
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RescoreSmem<KPT>& s = *reinterpret_cast<RescoreSmem<KPT>*>(smem_raw);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int b = blockIdx.y;
+  const RescoreJob job = p.job[blockIdx.z];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int C = visible_rows(p.n_rows, b, p.max_rows, p.status);
+  int ncb = p.cand_count[b];
+  if (ncb < 0 || ncb > p.cand_stride) {
+    set_status(p.status, ST_DEVICE_CHECK);
+    ncb = ncb < 0 ? 0 : p.cand_stride;
+  }
+  const int e0 = rank * EPC;  // first candidate of this CTA
+
+  for (int i = t; i < EPC / CSA2_BLK; i += RS_NT) {
+    const int cb = e0 / CSA2_BLK + i;
+    s.blocks[i] = cb < ncb ? p.cand[(int64_t)b * p.cand_stride + cb] : -1;
+  }
+  // B fragments: head n = lane / 4 (8 heads = MMA N), this thread's 16
+  // contiguous channels [16c, 16c + 16) of the 64, c = lane % 4.  The K axis
+  // is permuted identically for A and B so that each thread loads 32
+  // contiguous bytes of a row; a dot product does not depend on K order.
+  const int c = lane & 3, grp = lane >> 2;
+  uint32_t bq[8];
+  {
+    const uint4* qp = reinterpret_cast<const uint4*>(job.q_idx + ((int64_t)b * CSA2_HI + grp) *
+                                                                     CSA2_DI + 16 * c);
+    const uint4 q0 = __ldg(qp), q1 = __ldg(qp + 1);
+    bq[0] = q0.x; bq[1] = q0.y; bq[2] = q0.z; bq[3] = q0.w;
+    bq[4] = q1.x; bq[5] = q1.y; bq[6] = q1.z; bq[7] = q1.w;
+  }
+  const float w0 = __ldg(job.w + b * CSA2_HI + 2 * c), w1 = __ldg(job.w + b * CSA2_HI + 2 * c + 1);
+  __syncthreads();
+
+  // Score 16 candidates per warp step: rows grp and grp + 8 of the group.
+  for (int g = warp; g < EPC / 16; g += RS_NT / 32) {
+    uint32_t av[2][8];
+    bool valid[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int e = g * 16 + grp + 8 * h;  // candidate index within this CTA
+      const int blk = s.blocks[e / CSA2_BLK];
+      const int pos = blk * CSA2_BLK + (e % CSA2_BLK);
+      int64_t row = -1;
+      valid[h] = blk >= 0 && pos < C;
+      if (valid[h]) {
+        row = pos_row(p, b, pos);
+        if (row < 0) {
+          set_status(p.status, ST_DEVICE_CHECK);
+          valid[h] = false;
+        }
+      }
+      if (row >= 0) {
+        const uint4* kp = reinterpret_cast<const uint4*>(p.idx_k + row * CSA2_DI + 16 * c);
+        const uint4 k0 = __ldg(kp), k1 = __ldg(kp + 1);
+        av[h][0] = k0.x; av[h][1] = k0.y; av[h][2] = k0.z; av[h][3] = k0.w;
+        av[h][4] = k1.x; av[h][5] = k1.y; av[h][6] = k1.z; av[h][7] = k1.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; i++) av[h][i] = 0u;
+      }
+    }
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 4; ks++) {
+      const uint32_t a[4] = {av[0][2 * ks], av[1][2 * ks], av[0][2 * ks + 1], av[1][2 * ks + 1]};
+      mma_bf16_16816(d, a, bq[2 * ks], bq[2 * ks + 1]);
+    }
+    float s0 = fmaf(w1, fmaxf(d[1], 0.f), w0 * fmaxf(d[0], 0.f));
+    float s1 = fmaf(w1, fmaxf(d[3], 0.f), w0 * fmaxf(d[2], 0.f));
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+    if (c == 0) {
+      s.keys[g * 16 + grp] = valid[0] ? float_key(s0) : 0u;
+      s.keys[g * 16 + grp + 8] = valid[1] ? float_key(s1) : 0u;
+    }
+  }
+  __syncthreads();
+
+  uint32_t key[KPT];
+  int32_t id[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; j++) {
+    const int e = t * KPT + j;
+    key[j] = s.keys[e];
+    const int blk = s.blocks[e / CSA2_BLK];
+    id[j] = blk * CSA2_BLK + (e % CSA2_BLK);
+  }
+  cluster_select_topk<RS_NT, KPT>(s.sel, key, id, p.top_k,
+                                  job.idx + (int64_t)b * job.idx_stride, job.idx_count + b);
+}
+
+// --------------------------------------------- block Top-k (pool) select
+constexpr int BS_NT = 1024;
+constexpr int BS_KPT = 16;
+
+__global__ void __launch_bounds__(BS_NT) block_select_kernel(
+    const float* __restrict__ bm, int32_t bm_stride, const int32_t* __restrict__ n_rows,
+    int32_t max_rows, int32_t k_req, int32_t* sel, int32_t sel_stride, int32_t* sel_count,
+    uint32_t* status) {
+  __shared__ SelectSmem<BS_NT> sm;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int b = blockIdx.y;
+  const int C = visible_rows(n_rows, b, max_rows, status);
+  const int nblk = (C + CSA2_BLK - 1) / CSA2_BLK;
+  const int e0 = (rank * BS_NT + threadIdx.x) * BS_KPT;
+  uint32_t key[BS_KPT];
+  int32_t id[BS_KPT];
+  const float* src = bm + (int64_t)b * bm_stride + e0;
+#pragma unroll
+  for (int j = 0; j < BS_KPT; j += 4) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e0 + j < nblk) v = *reinterpret_cast<const float4*>(src + j);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      key[j + u] = (e0 + j + u < nblk) ? float_key(f[u]) : 0u;
+      id[j + u] = e0 + j + u;
+    }
+  }
+  cluster_select_topk<BS_NT, BS_KPT>(sm, key, id, k_req, sel + (int64_t)b * sel_stride,
+                                     sel_count + b);
+}
+
+// ------------------------------------------------------------ launchers
+cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
+                        int num_sms, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(score_scan_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
+  const int grid = (int)(total < 2LL * num_sms ? total : 2LL * num_sms);
+  if (grid <= 0) return cudaSuccess;
+  score_scan_kernel<<<grid, SC_THREADS, SC_SMEM, st>>>(map_k, map_q, p);
+  return cudaGetLastError();
+}
+
+template <int KPT>
+static cudaError_t launch_rescore_t(const RescoreParams& p, int n_jobs, int batch, int cs,
+                                    cudaStream_t st) {
+  auto kern = rescore_select_kernel<KPT>;
+  const size_t smem = sizeof(RescoreSmem<KPT>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  if (cs > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, batch, n_jobs);
+  cfg.blockDim = dim3(RS_NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// Candidates per sequence: n_cand_blocks * 8.  Picks a cluster of up to 16
+// CTAs of 256 threads holding 4 (else 16) candidates per thread.
+cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
+                           cudaStream_t st) {
+  const int ncand = n_cand_blocks * CSA2_BLK;
+  int cs = (ncand + RS_NT * 4 - 1) / (RS_NT * 4);
+  if (cs < 1) cs = 1;
+  if (cs <= 16) {
+    int c2 = 1;
+    while (c2 < cs) c2 <<= 1;
+    return launch_rescore_t<4>(p, n_jobs, batch, c2, st);
+  }
+  cs = (ncand + RS_NT * 16 - 1) / (RS_NT * 16);
+  int c2 = 1;
+  while (c2 < cs) c2 <<= 1;
+  if (c2 > 16) return cudaErrorInvalidValue;
+  return launch_rescore_t<16>(p, n_jobs, batch, c2, st);
+}
+
+cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n_rows,
+                                int max_rows, int batch, int k_req, int32_t* sel, int sel_stride,
+                                int32_t* sel_count, uint32_t* status, cudaStream_t st) {
+  const int nblk_max = (max_rows + CSA2_BLK - 1) / CSA2_BLK;
+  int cs = (nblk_max + BS_NT * BS_KPT - 1) / (BS_NT * BS_KPT);
+  if (cs < 1) cs = 1;
+  int c2 = 1;
+  while (c2 < cs) c2 <<= 1;
+  if (c2 > 8) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c2, batch, 1);
+  cfg.blockDim = dim3(BS_NT);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = c2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, block_select_kernel, bm, (int32_t)bm_stride, n_rows,
+                            (int32_t)max_rows, (int32_t)k_req, sel, (int32_t)sel_stride,
+                            sel_count, status);
+}
+
+}  // namespace csa2

@@ -1,0 +1,261 @@
+/*
+ * csa2.h -- C ABI of libcsa2.so: the CSA2 (Compressed Sparse Attention 2)
+ * decode step over an FP4 global KV cache, on one NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages on DeepSeek-V4.1-Flash), cited by tag:
+ *   [REL] "DeepSeek-V4.1-Flash 发布：100 万上下文 + FP4 KV Cache + 跨层注意力复用"
+ *         (feinterview.poetries.top)
+ *   [CNB] "DeepSeek V4.1 Flash 发布，百万上下文开始算缓存这笔账" (cnblogs, OpenCSG)
+ *   [YOM] yomxxx.com post on the V4.1-Flash CED/CSA2 paper (2026-09-14)
+ *   [TUC] "V4.1 Flash 内测，梁文锋又当回了梁圣" (tucaod.com; paper walk-through)
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer argument named as device memory must be a device pointer
+ *    of the current CUDA device; the caller allocates and owns every buffer.
+ *    The library allocates nothing, frees nothing and never synchronises,
+ *    except csa2_sync_status(), which exists to synchronise.
+ *  - All work is enqueued on the given stream and is asynchronous.
+ *  - Argument, shape and alignment errors are detected on the host and
+ *    returned before anything is launched.  Launch failures return
+ *    CSA2_ERR_CUDA.  Problems only the device can see (a page-table entry
+ *    outside the row pool, an expired bounded wait) never fault: the kernel
+ *    clamps, records a bit in the status word at the start of the workspace,
+ *    and csa2_sync_status() reports it as CSA2_ERR_DEVICE_CHECK or
+ *    CSA2_ERR_TIMEOUT.
+ *  - csa2_last_error() returns a thread-local message for the last failure.
+ *  - Device pointers must be 16-byte aligned (CSA2_ERR_ALIGNMENT otherwise).
+ *  - Shapes are fixed to the decode configuration of the pages and of the
+ *    synthetic workloads: main-KV rows of CSA2_D = 512 channels, CSA2_H = 16
+ *    query heads, an indexer of CSA2_HI = 8 heads x CSA2_DI = 64, blocks of
+ *    CSA2_BLK = 8 positions, a sliding window of CSA2_W = 128 rows.
+ */
+#ifndef CSA2_API_H_
+#define CSA2_API_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csa2_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+enum {
+  CSA2_D = 512,          /* main-KV channels per entry                         */
+  CSA2_H = 16,           /* query heads sharing one main-KV row (K = V)        */
+  CSA2_HI = 8,           /* indexer heads                                      */
+  CSA2_DI = 64,          /* indexer head dimension                             */
+  CSA2_BLK = 8,          /* positions per HSI block [YOM §二 HSI]              */
+  CSA2_W = 128,          /* sliding-window rows [REL §CED; YOM §一]            */
+  CSA2_MAX_TOPK = 512,   /* Top-512 [REL §CSA2; YOM §二 table]                 */
+  CSA2_MAX_POOL = 2048,  /* 2,048 blocks = 16,384 positions [YOM §二 HSI]      */
+  CSA2_MAX_ROWS = 1 << 20 /* visible entries per sequence (1M context)        */
+};
+
+typedef enum {
+  CSA2_OK = 0,
+  CSA2_ERR_INVALID_ARG = 1,  /* NULL pointer, bad enum, bad count              */
+  CSA2_ERR_SHAPE = 2,        /* a size outside what the kernels support        */
+  CSA2_ERR_ALIGNMENT = 3,    /* a pointer not 16-byte aligned                  */
+  CSA2_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required        */
+  CSA2_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed           */
+  CSA2_ERR_TIMEOUT = 6,      /* a device-side bounded wait expired             */
+  CSA2_ERR_DEVICE_CHECK = 7  /* a device-side bounds check clamped an index    */
+} csa2_status;
+
+typedef enum { CSA2_FULL = 0, CSA2_REINDEX = 1, CSA2_REUSE = 2 } csa2_mode;
+
+/*
+ * FP4 main-KV cache, E2M1 values with one E4M3 scale per 16 channels and no
+ * global scale ("NVFP4 without its global scale") [REL §FP4 KV; YOM §三;
+ * TUC §缓存精度与持久化分层], stored as two planes over a pool of rows:
+ *   codes  [pool_rows][CSA2_D/2]  two E2M1 codes per byte, even channel in
+ *                                 the low nibble
+ *   scales [pool_rows][CSA2_D/16] E4M3 bit patterns
+ *   idx_k  [pool_rows][CSA2_DI]   bf16 indexer K of each row, projected from
+ *                                 the main-KV entry [YOM §二 last paragraph]
+ * Position p (0 <= p < n_rows[b]) of sequence b is pool row
+ *   page_table == NULL: b * seq_stride + p
+ *   otherwise:          page_table[b * max_pages + p / page_rows] * page_rows
+ *                       + p % page_rows      (page_rows must be 64)
+ * A row outside [0, pool_rows) is never dereferenced: it reads as zeros and
+ * sets CSA2_ERR_DEVICE_CHECK.  All pointers are device pointers.
+ */
+typedef struct {
+  const uint8_t *codes;
+  const uint8_t *scales;
+  const uint16_t *idx_k;
+  const int32_t *page_table; /* [batch][max_pages] or NULL                     */
+  int32_t page_rows;         /* 64 when paged, ignored otherwise               */
+  int32_t max_pages;
+  const int32_t *n_rows;     /* [batch] visible entries C_b (device)           */
+  int32_t batch;
+  int32_t max_rows;          /* host upper bound of every n_rows[b]            */
+  int64_t seq_stride;        /* contiguous layout only                         */
+  int64_t pool_rows;
+} csa2_kv_view;
+
+/* ---------------------------------------------------------------- status */
+
+const char *csa2_status_string(csa2_status s);
+/* Thread-local text of the last error returned on this thread ("" if none). */
+const char *csa2_last_error(void);
+
+/* Bytes at the start of every workspace that hold the device status word. */
+#define CSA2_WS_HEADER 256
+/* Zero the status word of a workspace (enqueued on stream).  Call once
+ * before the first use of a workspace. */
+csa2_status csa2_workspace_init(void *ws, size_t ws_bytes, csa2_stream_t stream);
+/* Synchronise the stream, read and clear the status word: CSA2_OK, or the
+ * first device-side problem recorded since the last call. */
+csa2_status csa2_sync_status(void *ws, csa2_stream_t stream);
+
+/* ---------------------------------------------------------------- tracing */
+
+/*
+ * Optional per-launch timing.  While a trace is set on the calling thread,
+ * every entry point records trace->events[trace->count] (a cudaEvent_t the
+ * caller created with timing enabled) on its stream just before each kernel
+ * launch, with the kernel's stage name in trace->names[], and one event named
+ * "end" after its last launch; count advances by one per event and recording
+ * stops silently at capacity (at most 64).  Stage i lasts from event i to
+ * event i+1.  NULL turns tracing off.  Tracing adds event records only.
+ */
+typedef struct {
+  void *events[64];
+  const char *names[64];
+  int32_t capacity;
+  int32_t count;
+} csa2_trace;
+void csa2_trace_set(csa2_trace *trace);
+
+/* ------------------------------------------------------------- FP4 codec */
+
+/*
+ * Quantise rows of bf16 values x[rows][ch] (ch a multiple of 16) to the FP4
+ * planes codes[rows][ch/2] and scales[rows][ch/16] [REL §FP4 KV; YOM §三].
+ * Per group of 16: amax = max|x|; t = amax / 6 in fp32 (correctly rounded);
+ * scale = E4M3(t) round-to-nearest-even, saturating at 448; a zero scale
+ * gives all codes 0x0; otherwise code_i = E2M1(x_i / scale), nearest-even,
+ * saturating at 6, sign kept (a negative value that rounds to zero is 0x8).
+ * Inputs must be finite.  rows may be 0.  Device pointers.
+ */
+csa2_status csa2_quantize_fp4(const uint16_t *x_bf16, int64_t rows, int32_t ch,
+                              uint8_t *codes, uint8_t *scales, csa2_stream_t stream);
+
+/* y[rows][ch] = bf16(e2m1(code) * e4m3(scale)); exact (every product is a
+ * bf16 value).  Device pointers. */
+csa2_status csa2_dequantize_fp4(const uint8_t *codes, const uint8_t *scales, int64_t rows,
+                                int32_t ch, uint16_t *y_bf16, csa2_stream_t stream);
+
+/* ------------------------------------------------------------ the indexer */
+
+/*
+ * Workspace bytes csa2_index_full / csa2_index_reindex need for this view.
+ */
+size_t csa2_index_workspace_size(const csa2_kv_view *kv, int32_t top_k, int32_t pool_blocks);
+
+/*
+ * Full-mode indexer [REL §CSA2 "Full"; YOM §二 mode table and HSI paragraph;
+ * TUC §CSA2注意力].  For every sequence b, over all visible positions p < C_b:
+ *   s[p] = sum_h w[b][h] * max(0, q_idx[b][h] . idx_k[row(b,p)])
+ * (the score form is this library's reading; the pages only say "score"),
+ * block maxima over blocks of CSA2_BLK positions, and
+ *   pool[b][0..pool_count[b])  the min(pool_blocks, ceil(C_b/8)) blocks with
+ *                              the largest block maxima, ascending block ids
+ *                              (the decoder Hierarchical Sparse Indexer pool)
+ *   idx[b][0..idx_count[b])    the min(top_k, C_b) positions with the largest
+ *                              s, ascending, ties to the lower position
+ * Entries past the counts are -1.  pool_blocks = 0 builds no pool (pool and
+ * pool_count may be NULL).  top_k in [1, 512]; pool_blocks in {0} or
+ * [top_k ... 2048].  q_idx: bf16 [batch][8][64]; w: fp32 [batch][8];
+ * idx: int32 [batch][top_k]; pool: int32 [batch][pool_blocks].  Device.
+ */
+csa2_status csa2_index_full(const csa2_kv_view *kv, const uint16_t *q_idx, const float *w,
+                            int32_t top_k, int32_t pool_blocks, int32_t *idx,
+                            int32_t *idx_count, int32_t *pool, int32_t *pool_count,
+                            void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/*
+ * Reindex-mode indexer [REL §CSA2 "Reindex"; YOM §二 table: reuses the Full
+ * layer's main KV and indexer K, rescores with its own indexer query].
+ * With a pool (pool != NULL) only the positions of the pool blocks are
+ * rescored [YOM §二 HSI: later indexers search only inside the pool]; with
+ * pool == NULL every visible position is.  Output as csa2_index_full.
+ * pool: int32 [batch][pool_stride] ascending block ids, pool_count [batch].
+ */
+csa2_status csa2_index_reindex(const csa2_kv_view *kv, const uint16_t *q_idx, const float *w,
+                               const int32_t *pool, const int32_t *pool_count,
+                               int32_t pool_stride, int32_t top_k, int32_t *idx,
+                               int32_t *idx_count, void *ws, size_t ws_bytes,
+                               csa2_stream_t stream);
+
+/* ---------------------------------------------------------- the attention */
+
+size_t csa2_attn_workspace_size(int32_t batch, int32_t n_layers);
+
+/*
+ * Sparse + sliding-window decode attention of one layer [TUC core-attention
+ * figure text: Selection / Top-K / Concatenation; REL §CED: 128-token SWA at
+ * every layer with FP8 KV].  For each sequence b and head h:
+ *   keys = values = [ dequant(main KV at idx[b][0..idx_count[b]) ) ;
+ *                     E4M3 window swa[b][0..swa_len[b]) ]
+ *   out[b][h] = softmax_j(sm_scale * q[b][h] . key_j) . values
+ * one softmax over both branches (MQA: the 16 heads share each row as K and
+ * V).  No keys gives zeros.  q: bf16 [batch][16][512] (|q| < 65504);
+ * idx: int32 [batch][idx_stride]; swa: uint8 E4M3 [batch][128][512];
+ * swa_len: int32 [batch] (<= 128); out: bf16 [batch][16][512].  Device.
+ */
+csa2_status csa2_sparse_attn_decode(const uint16_t *q, const csa2_kv_view *kv,
+                                    const int32_t *idx, const int32_t *idx_count,
+                                    int32_t idx_stride, const uint8_t *swa,
+                                    const int32_t *swa_len, float sm_scale, uint16_t *out,
+                                    void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* ---------------------------------------------------------- a layer group */
+
+/*
+ * One decode step of a group of CSA2 layers sharing one main-KV cache
+ * [REL §CSA2; YOM §二: layers statically Full, Reindex or Reuse; every layer
+ * keeps its own query and SWA KV; decoder = Full+3 Reuse, then 4 x
+ * (Reindex+3 Reuse)].  Layer 0 must be FULL.  A REINDEX layer rescores the
+ * pool of the latest FULL layer (all positions when pool_blocks == 0).  A
+ * REUSE layer takes the latest FULL/REINDEX indices unchanged.
+ * Per-layer inputs are stacked on a leading layer axis:
+ *   q_idx bf16 [L][batch][8][64], w fp32 [L][batch][8] (read for FULL and
+ *   REINDEX layers only), q bf16 [L][batch][16][512],
+ *   swa E4M3 [L][batch][128][512], swa_len int32 [batch].
+ * Outputs: idx int32 [L][batch][top_k] and idx_count [L][batch] (REUSE layers
+ * receive a copy of the indices they used), pool int32 [batch][pool_blocks]
+ * and pool_count [batch] of the last FULL layer (may be NULL when
+ * pool_blocks == 0), out bf16 [L][batch][16][512].
+ * modes points to HOST memory; everything else is device memory.
+ */
+typedef struct {
+  csa2_kv_view kv;
+  int32_t n_layers;
+  const int32_t *modes; /* host [n_layers] */
+  const uint16_t *q_idx;
+  const float *w;
+  const uint16_t *q;
+  const uint8_t *swa;
+  const int32_t *swa_len;
+  int32_t top_k;
+  int32_t pool_blocks;
+  float sm_scale;
+  int32_t *idx;
+  int32_t *idx_count;
+  int32_t *pool;
+  int32_t *pool_count;
+  uint16_t *out;
+} csa2_group_desc;
+
+size_t csa2_group_workspace_size(const csa2_group_desc *desc);
+csa2_status csa2_layer_group(const csa2_group_desc *desc, void *ws, size_t ws_bytes,
+                             csa2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_API_H_ */
