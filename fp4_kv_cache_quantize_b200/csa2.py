@@ -82,6 +82,8 @@ _dequantize = _sig("csa2_dequantize_fp4", C.c_int, [_vp, _vp, _i64, _i32, _vp, _
 _index_ws = _sig("csa2_index_workspace_size", _sz, [C.POINTER(KVView), _i32, _i32])
 _index_full = _sig("csa2_index_full", C.c_int,
                    [C.POINTER(KVView), _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_index_full_noalloc = _sig("csa2_index_full_noalloc", C.c_int,
+                           [C.POINTER(KVView), _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp])
 _index_reindex = _sig("csa2_index_reindex", C.c_int,
                       [C.POINTER(KVView), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _sz,
                        _vp])
@@ -173,6 +175,15 @@ def csa2_index_full(kv: KVCache, q_idx, w, top_k, pool_blocks, idx, idx_count, p
     _check(_index_full(C.byref(kv.view), _ptr(q_idx), _ptr(w), top_k, pool_blocks, _ptr(idx),
                        _ptr(idx_count), _ptr(pool), _ptr(pool_count), _ptr(ws), ws.numel(),
                        _stream(stream)))
+
+
+def csa2_index_full_noalloc(kv: KVCache, q_idx, w, top_k, pool_blocks, idx, idx_count, pool,
+                            pool_count, stream=None):
+    """csa2_index_full with the library's static scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _check(_index_full_noalloc(C.byref(kv.view), _ptr(q_idx), _ptr(w), top_k, pool_blocks,
+                               _ptr(idx), _ptr(idx_count), _ptr(pool), _ptr(pool_count),
+                               _stream(stream)))
 
 
 def csa2_index_reindex(kv: KVCache, q_idx, w, pool, pool_count, pool_stride, top_k, idx,

@@ -1,0 +1,63 @@
+// noalloc.cu -- csa2_index_full_noalloc: the Full-mode indexer for callers
+// that cannot allocate device memory.
+//
+// Its scratch (status word, block maxima, candidate blocks) is a file-scope
+// static __device__ array of CSA2_NOALLOC_SCRATCH_BYTES that every GPU which
+// loads this library holds until the process exits.  Host code must not pass
+// the array's name to a kernel: on the host that name is a stand-in, not a
+// device address.  The device address is looked up once per device with
+// cudaGetSymbolAddress (on that device's first call) and handed to the same
+// code path as csa2_index_full with a caller workspace.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "capi_common.h"
+
+namespace csa2 {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[CSA2_NOALLOC_SCRATCH_BYTES];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[256];  // per device ordinal
+
+// Device address of the static scratch on the current device.
+static csa2_status noalloc_scratch(void** out) {
+  int dev = 0;
+  CSA2_CUDA(cudaGetDevice(&dev));
+  CSA2_REQUIRE(dev >= 0 && dev < 256, CSA2_ERR_INVALID_ARG, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CSA2_OK;
+}
+
+}  // namespace csa2
+
+extern "C" csa2_status csa2_index_full_noalloc(const csa2_kv_view* kv, const uint16_t* q_idx,
+                                               const float* w, int32_t top_k,
+                                               int32_t pool_blocks, int32_t* idx,
+                                               int32_t* idx_count, int32_t* pool,
+                                               int32_t* pool_count, csa2_stream_t stream) {
+  using namespace csa2;
+  CSA2_REQUIRE(kv != nullptr, CSA2_ERR_INVALID_ARG, "kv is NULL");
+  const size_t need = csa2_index_workspace_size(kv, top_k, pool_blocks);
+  CSA2_REQUIRE(need > 0, CSA2_ERR_SHAPE, "top_k = %d is not a valid Top-k size", top_k);
+  CSA2_REQUIRE(need <= (size_t)CSA2_NOALLOC_SCRATCH_BYTES, CSA2_ERR_WORKSPACE,
+               "this batch and context need %zu bytes of scratch but the static scratch holds "
+               "%u; use csa2_index_full with a caller workspace",
+               need, (unsigned)CSA2_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  csa2_status r = noalloc_scratch(&scratch);
+  if (r) return r;
+  // The status word must start at zero; everything else in the scratch is
+  // written before it is read.
+  CSA2_CUDA(cudaMemsetAsync(scratch, 0, CSA2_WS_HEADER, (cudaStream_t)stream));
+  return csa2_index_full(kv, q_idx, w, top_k, pool_blocks, idx, idx_count, pool, pool_count,
+                         scratch, (size_t)CSA2_NOALLOC_SCRATCH_BYTES, stream);
+}

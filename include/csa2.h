@@ -191,6 +191,36 @@ csa2_status csa2_index_reindex(const csa2_kv_view *kv, const uint16_t *q_idx, co
                                int32_t *idx_count, void *ws, size_t ws_bytes,
                                csa2_stream_t stream);
 
+/*
+ * csa2_index_full without any device allocation by the caller.  The pages
+ * have no counterpart: this is an integration convenience.  It is for callers
+ * that cannot allocate device memory while they run -- plugins or custom ops
+ * inside a host framework that owns all device memory through its own
+ * allocator, serving loops that must not pay cudaMalloc's implicit device
+ * synchronisation, processes already at their memory limit.
+ *
+ * Same arguments, checks and outputs as csa2_index_full, minus the
+ * workspace.  Its scratch is one static device array of
+ * CSA2_NOALLOC_SCRATCH_BYTES (2 MiB) inside libcsa2.so, which every GPU that
+ * loads the library holds until the process exits.  A batch and context
+ * needing more scratch than that (csa2_index_workspace_size() larger than
+ * CSA2_NOALLOC_SCRATCH_BYTES; e.g. batch x ceil(context / 8) x 4 bytes above
+ * about 2 MB) is rejected with CSA2_ERR_WORKSPACE before any launch.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array: calls whose work overlaps on the GPU
+ * (two streams, two threads) race and must be serialised by the caller.
+ * Device-side range checks still clamp, but their status bit stays in the
+ * shared scratch (cleared at the start of each call) and is not reported;
+ * use csa2_index_full with csa2_sync_status to diagnose such inputs.
+ * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (2u << 20)
+csa2_status csa2_index_full_noalloc(const csa2_kv_view *kv, const uint16_t *q_idx,
+                                    const float *w, int32_t top_k, int32_t pool_blocks,
+                                    int32_t *idx, int32_t *idx_count, int32_t *pool,
+                                    int32_t *pool_count, csa2_stream_t stream);
+
 /* ---------------------------------------------------------- the attention */
 
 size_t csa2_attn_workspace_size(int32_t batch, int32_t n_layers);
