@@ -13,12 +13,17 @@
 // swizzled shared tile (E2M1 x E4M3 and E4M3 are exact in fp16), computes
 // S = Q K^T and O += P V with m16n8k16 tensor-core tiles (M = the 16 heads:
 // a per-step tile far too small for tcgen05's 64/128-row MMA), keeps the
-// online-softmax state in fp32, and either normalises or writes a partial
-// (O, max, sum) for attn_merge_kernel.
+// online-softmax state in fp32.  The CTAs of one (layer, sequence) form a
+// thread-block cluster: at the end each publishes its unnormalised O, max and
+// sum in shared memory and the cluster merges them through distributed
+// shared memory (log-sum-exp weights), each CTA finishing a slice of the
+// output.  No partial result goes to HBM and no second kernel runs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
+
+#include <cooperative_groups.h>
 
 #include "csa2_internal.cuh"
 #include "kernels.h"
@@ -38,6 +43,9 @@ struct AttnSmem {
   __half p[CSA2_H * AT_CH];    // swizzled rows of 128 B
   float s[CSA2_H][AT_CH + 4];
   float m[CSA2_H], l[CSA2_H], alpha[CSA2_H];
+  float mall[16][CSA2_H], lall[16][CSA2_H];  // split merge: every rank's max and sum
+  float fr[16][CSA2_H];                      // weight of each rank's partial
+  float invl[CSA2_H];
   int64_t row[AT_CH];
 };
 
@@ -87,6 +95,7 @@ __device__ __forceinline__ int64_t kv_row(const AttnParams& p, int b, int pos) {
 __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   AttnSmem& s = *reinterpret_cast<AttnSmem*>(smem_raw);
+  pdl_wait();  // the indices come from the previous kernel
   const int split = blockIdx.x, b = blockIdx.y, li = blockIdx.z;
   const AttnLayer L = p.layer[li];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -116,25 +125,33 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
     if (t == 0) L.idx_copy_count[b] = L.idx_count[b];
   }
 
-  // Q: bf16 -> fp16 (|q| < 65504 required), swizzled rows.
+  // Q (bf16) is loaded now and converted to fp16 (|q| < 65504 required) into
+  // swizzled rows once the first chunk's gathers are in flight.
+  constexpr int QV = (CSA2_H * CSA2_D / 8) / AT_NT;
+  uint4 qv[QV];
   {
     const uint4* qg = reinterpret_cast<const uint4*>(L.q + (int64_t)b * CSA2_H * CSA2_D);
 #pragma unroll
-    for (int u = 0; u < (CSA2_H * CSA2_D / 8) / AT_NT; u++) {
+    for (int u = 0; u < QV; u++) qv[u] = __ldg(qg + t + u * AT_NT);
+  }
+  bool q_ready = false;
+  auto store_q = [&]() {
+#pragma unroll
+    for (int u = 0; u < QV; u++) {
       const int i = t + u * AT_NT;  // 16-byte chunk of 8 channels
       const int row = i >> 6, ch = i & 63;
-      const uint4 v = __ldg(qg + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t o[4];
+      const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+      uint32_t o4[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) {
         const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
-        o[k] = h2_bits(__floats2half2_rn(lo, hi));
+        o4[k] = h2_bits(__floats2half2_rn(lo, hi));
       }
       *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(s.q) + sw1024(row, ch)) =
-          make_uint4(o[0], o[1], o[2], o[3]);
+          make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
-  }
+    q_ready = true;
+  };
   if (t < CSA2_H) {
     s.m[t] = -INFINITY;
     s.l[t] = 0.0f;
@@ -181,20 +198,23 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
           sv[u] = 0;
         }
       }
+      if (!q_ready) store_q();
 #pragma unroll
       for (int u = 0; u < 8; u++) {
         const int i = t + u * AT_NT, r = i >> 4, cc = i & 15;
         const __half s0 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sv[u] & 0xFF), __NV_E4M3));
         const __half s1 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sv[u] >> 8), __NV_E4M3));
-        const uint32_t wv[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
 #pragma unroll
-        for (int q4 = 0; q4 < 4; q4++) {  // 4 bytes of codes = 8 channels
+        for (int q4i = 0; q4i < 4; q4i++) {  // 4 bytes of codes = 8 channels
+          // rotate by cc so that one store instruction spreads over all banks
+          const int q4 = (q4i + cc) & 3;
+          const uint32_t word = q4 == 0 ? cv[u].x : q4 == 1 ? cv[u].y : q4 == 2 ? cv[u].z : cv[u].w;
           const __half2 sc = q4 < 2 ? __half2(s0, s0) : __half2(s1, s1);
           uint32_t hv[4];
 #pragma unroll
           for (int k = 0; k < 4; k++) {
             const __half2 v = __half2(__nv_cvt_fp4x2_to_halfraw2(
-                (__nv_fp4x2_storage_t)((wv[q4] >> (8 * k)) & 0xFF), __NV_E2M1));
+                (__nv_fp4x2_storage_t)((word >> (8 * k)) & 0xFF), __NV_E2M1));
             hv[k] = h2_bits(__hmul2(v, sc));
           }
           *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(s.kv) + sw1024(r, cc * 4 + q4)) =
@@ -212,6 +232,7 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
         cv[u] = row >= 0 ? __ldg(reinterpret_cast<const uint4*>(swa + row * CSA2_D) + cc)
                          : make_uint4(0, 0, 0, 0);
       }
+      if (!q_ready) store_q();
 #pragma unroll
       for (int u = 0; u < 16; u++) {
         const int i = t + u * AT_NT, r = i >> 5, cc = i & 31;
@@ -225,9 +246,11 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
               (__nv_fp8x2_storage_t)(wv[k] >> 16), __NV_E4M3)));
         }
         uint8_t* base = reinterpret_cast<uint8_t*>(s.kv);
-        *reinterpret_cast<uint4*>(base + sw1024(r, 2 * cc)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        *reinterpret_cast<uint4*>(base + sw1024(r, 2 * cc + 1)) =
-            make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        const uint4 lo = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        const uint4 hi = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        const int odd = cc & 1;  // alternate the order across lanes (bank spread)
+        *reinterpret_cast<uint4*>(base + sw1024(r, 2 * cc + odd)) = odd ? hi : lo;
+        *reinterpret_cast<uint4*>(base + sw1024(r, 2 * cc + 1 - odd)) = odd ? lo : hi;
       }
     }
     __syncthreads();
@@ -328,11 +351,10 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
   }
   __syncthreads();
 
-  const int64_t pair = (int64_t)li * p.batch + b;
+  uint16_t* out = L.out + (int64_t)b * CSA2_H * CSA2_D;
   if (p.nsplit == 1) {
     const float l0 = s.l[g], l1 = s.l[g + 8];
     const float inv0 = l0 > 0.f ? 1.0f / l0 : 0.f, inv1 = l1 > 0.f ? 1.0f / l1 : 0.f;
-    uint16_t* out = L.out + (int64_t)b * CSA2_H * CSA2_D;
 #pragma unroll
     for (int nt = 0; nt < 16; nt++) {
       const int ch = warp * 128 + nt * 8 + 2 * tig;
@@ -341,47 +363,64 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
       *reinterpret_cast<__nv_bfloat162*>(out + g * CSA2_D + ch) = r0;
       *reinterpret_cast<__nv_bfloat162*>(out + (g + 8) * CSA2_D + ch) = r1;
     }
-  } else {
-    float* po = p.part_o + (pair * p.nsplit + split) * CSA2_H * CSA2_D;
-#pragma unroll
-    for (int nt = 0; nt < 16; nt++) {
-      const int ch = warp * 128 + nt * 8 + 2 * tig;
-      *reinterpret_cast<float2*>(po + g * CSA2_D + ch) = make_float2(o[nt][0], o[nt][1]);
-      *reinterpret_cast<float2*>(po + (g + 8) * CSA2_D + ch) = make_float2(o[nt][2], o[nt][3]);
-    }
-    if (t < CSA2_H) {
-      float* ml = p.part_ml + ((pair * p.nsplit + split) * CSA2_H + t) * 2;
-      ml[0] = s.m[t];
-      ml[1] = s.l[t];
+    return;
+  }
+  // Split merge across the cluster, push-only: after every rank has finished
+  // with its key/value tile, each rank writes its (max, sum) to every rank and
+  // each pair of its unnormalised O to the rank that owns that pair of output
+  // elements (into the owner's idle key/value tile); after a second cluster
+  // barrier every rank reduces its own slice from local shared memory.
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int ns = p.nsplit;
+  const int rank = (int)cluster.block_rank();
+  constexpr int NPAIR = CSA2_H * CSA2_D / 2;
+  const int slice = (NPAIR + ns - 1) / ns + 1;  // receive row length in pairs
+  cluster.sync();  // every rank is done with its key/value tile
+  if (t < CSA2_H) {
+    for (int r = 0; r < ns; r++) {
+      *cluster.map_shared_rank(&s.mall[rank][t], r) = s.m[t];
+      *cluster.map_shared_rank(&s.lall[rank][t], r) = s.l[t];
     }
   }
-}
-
-// Combine the split partials of one (layer, sequence): log-sum-exp merge.
-__global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p) {
-  const int b = blockIdx.x, li = blockIdx.y;
-  const int64_t pair = (int64_t)li * p.batch + b;
-  const float* po = p.part_o + pair * p.nsplit * CSA2_H * CSA2_D;
-  const float* ml = p.part_ml + pair * p.nsplit * CSA2_H * 2;
-  uint16_t* out = p.layer[li].out + (int64_t)b * CSA2_H * CSA2_D;
-  for (int i = threadIdx.x * 2; i < CSA2_H * CSA2_D; i += 512) {
-    const int h = i / CSA2_D;
-    float mx = -INFINITY;
-    for (int sp = 0; sp < p.nsplit; sp++) mx = fmaxf(mx, ml[(sp * CSA2_H + h) * 2]);
-    float den = 0.f, n0 = 0.f, n1 = 0.f;
-    if (mx != -INFINITY) {
-      for (int sp = 0; sp < p.nsplit; sp++) {
-        const float m = ml[(sp * CSA2_H + h) * 2];
-        if (m == -INFINITY) continue;
-        const float f = exp2f(m - mx);
-        den += ml[(sp * CSA2_H + h) * 2 + 1] * f;
-        const float2 v = *reinterpret_cast<const float2*>(po + (int64_t)sp * CSA2_H * CSA2_D + i);
-        n0 += v.x * f;
-        n1 += v.y * f;
-      }
+#pragma unroll
+  for (int nt = 0; nt < 16; nt++) {
+#pragma unroll
+    for (int hh = 0; hh < 2; hh++) {
+      const int row = g + 8 * hh;
+      const int q = (row * CSA2_D + warp * 128 + nt * 8 + 2 * tig) >> 1;  // pair index
+      const int owner = ((q + 1) * ns - 1) / NPAIR;
+      const int q0 = owner * NPAIR / ns;
+      float2* dst = reinterpret_cast<float2*>(s.kv) + rank * slice + (q - q0);
+      *cluster.map_shared_rank(dst, owner) = make_float2(o[nt][2 * hh], o[nt][2 * hh + 1]);
     }
-    const float inv = den > 0.f ? 1.0f / den : 0.f;
-    *reinterpret_cast<__nv_bfloat162*>(out + i) = __floats2bfloat162_rn(n0 * inv, n1 * inv);
+  }
+  cluster.sync();  // all pushes have landed; no remote access after this
+  if (t < CSA2_H) {
+    float mx = -INFINITY;
+    for (int r = 0; r < ns; r++) mx = fmaxf(mx, s.mall[r][t]);
+    float den = 0.f;
+    for (int r = 0; r < ns; r++) {
+      const float mr = s.mall[r][t];
+      const float f = (mx == -INFINITY || mr == -INFINITY) ? 0.f : exp2f(mr - mx);
+      s.fr[r][t] = f;
+      den += f * s.lall[r][t];
+    }
+    s.invl[t] = den > 0.f ? 1.0f / den : 0.f;
+  }
+  __syncthreads();
+  const int q0 = rank * NPAIR / ns, q1 = (rank + 1) * NPAIR / ns;
+  const float2* recv = reinterpret_cast<const float2*>(s.kv);
+  for (int q = q0 + t; q < q1; q += AT_NT) {
+    const int h = (2 * q) / CSA2_D;
+    float a0 = 0.f, a1 = 0.f;
+    for (int r = 0; r < ns; r++) {
+      const float2 v = recv[r * slice + (q - q0)];
+      a0 = fmaf(s.fr[r][h], v.x, a0);
+      a1 = fmaf(s.fr[r][h], v.y, a1);
+    }
+    *reinterpret_cast<__nv_bfloat162*>(out + 2 * q) =
+        __floats2bfloat162_rn(a0 * s.invl[h], a1 * s.invl[h]);
   }
 }
 
@@ -399,21 +438,27 @@ cudaError_t launch_attn(const AttnParams& p, cudaStream_t st) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(AttnSmem));
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
     attr_done = true;
   }
   trace_mark("attn", st);
-  attn_decode_kernel<<<dim3(p.nsplit, p.batch, p.n_layers), AT_NT, sizeof(AttnSmem), st>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || p.nsplit == 1) return e;
-  trace_mark("attn_merge", st);
-  attn_merge_kernel<<<dim3(p.batch, p.n_layers), 256, 0, st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.nsplit, p.batch, p.n_layers);
+  cfg.blockDim = dim3(AT_NT);
+  cfg.dynamicSmemBytes = sizeof(AttnSmem);
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = p.nsplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, attn_decode_kernel, p);
 }
 
-size_t attn_partial_bytes(int batch, int n_layers, int nsplit) {
-  if (nsplit <= 1) return 0;
-  const size_t pairs = (size_t)batch * n_layers * nsplit;
-  return pairs * CSA2_H * CSA2_D * sizeof(float) + pairs * CSA2_H * 2 * sizeof(float);
-}
 
 }  // namespace csa2

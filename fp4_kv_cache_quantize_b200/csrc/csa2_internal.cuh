@@ -162,6 +162,18 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while
+// its predecessor in the stream still runs; it must execute pdl_wait() before
+// reading anything the predecessor writes (the wait returns once the
+// predecessor has completed and its memory is visible).  Every CTA of a
+// predecessor calls pdl_launch_dependents() on entry, so the dependent grid is
+// scheduled only once all of the predecessor's CTAs are resident.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ misc
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

@@ -27,7 +27,8 @@ namespace csa2 {
 // ------------------------------------------------------------- the scan
 constexpr int SC_BOX = 64;                 // rows per TMA box
 constexpr int SC_N = 16;                   // indexer heads padded to MMA N
-constexpr int SC_STAGES = 5;
+constexpr int SC_STAGES = 6;
+constexpr int SC_ACC = 4;                  // TMEM accumulator buffers (16 columns each)
 constexpr int SC_A_BYTES = SC_TILE * 128;  // 16 KB of indexer K per stage
 constexpr int SC_B_BYTES = SC_N * 128;     // 2 KB of indexer query per stage
 constexpr int SC_THREADS = 192;            // producer, MMA, 4 epilogue warps
@@ -37,7 +38,7 @@ struct ScanSmem {
   uint8_t a[SC_STAGES][SC_A_BYTES];
   uint8_t b[SC_STAGES][SC_B_BYTES];
   uint64_t full[SC_STAGES], empty[SC_STAGES];
-  uint64_t tfull[2], tempty[2], done;
+  uint64_t tfull[SC_ACC], tempty[SC_ACC], done;
   uint32_t tmem_base;
   int abort;
 };
@@ -81,13 +82,14 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
   const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SC_STAGES; i++) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int i = 0; i < 2; i++) {
+    for (int i = 0; i < SC_ACC; i++) {
       mbar_init(&s.tfull[i], 1);
       mbar_init(&s.tempty[i], 4 * 32);
     }
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     tma_prefetch_desc(&map_q);
   }
   if (warp == 1) {
-    tmem_alloc(&s.tmem_base, 32);  // two 16-column fp32 accumulators
+    tmem_alloc(&s.tmem_base, SC_ACC * SC_N);  // SC_ACC 16-column fp32 accumulators
     tmem_relinquish();
   }
   tc_fence_before();
@@ -109,11 +111,14 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {  // ---------------------------------- TMA producer
-      int stage = 0;
+      int stage = 0, cur_b = -1, C = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
       for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
         const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
-        const int C = visible_rows(p.n_rows, b, p.max_rows, p.status);
+        if (b != cur_b) {
+          C = visible_rows(p.n_rows, b, p.max_rows, p.status);
+          cur_b = b;
+        }
         if (t * SC_TILE >= C) continue;
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort)) {
           s.abort = 1;
@@ -142,11 +147,14 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------------------------- MMA issuer
-      int stage = 0, acc = 0;
+      int stage = 0, acc = 0, cur_b = -1, C = 0;
       uint32_t phase = 0, acc_phase = 0;
       for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
         const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
-        const int C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
+        if (b != cur_b) {
+          C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
+          cur_b = b;
+        }
         if (t * SC_TILE >= C) continue;
         if (!mbar_wait(&s.full[stage], phase, abort) ||
             !mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort)) {
@@ -167,8 +175,10 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
           stage = 0;
           phase ^= 1u;
         }
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == SC_ACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       umma_commit(&s.done);  // completes once every MMA issued above has
       if (!mbar_wait(&s.done, 0, nullptr)) set_status(p.status, ST_TIMEOUT);
@@ -178,11 +188,16 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    int cur_b = -1;
+    int cur_b = -1, C = 0;
     float w[CSA2_HI];
     for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
       const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
-      const int C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
+      if (b != cur_b) {
+        C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
+#pragma unroll
+        for (int h = 0; h < CSA2_HI; h++) w[h] = __ldg(p.w + b * CSA2_HI + h);
+        cur_b = b;
+      }
       if (t * SC_TILE >= C) continue;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.tfull[acc], acc_phase, abort));
       if (!ok) {
@@ -196,11 +211,6 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
-      if (b != cur_b) {
-#pragma unroll
-        for (int h = 0; h < CSA2_HI; h++) w[h] = __ldg(p.w + b * CSA2_HI + h);
-        cur_b = b;
-      }
       float sc = 0.0f;
 #pragma unroll
       for (int h = 0; h < CSA2_HI; h++) sc = fmaf(w[h], fmaxf(__uint_as_float(r[h]), 0.0f), sc);
@@ -210,28 +220,33 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
       sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
       sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
       if ((lane & 7) == 0 && pos < C) p.bm[(int64_t)b * p.bm_stride + pos / CSA2_BLK] = sc;
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == SC_ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, SC_ACC * SC_N);
   }
 }
 
 // ------------------------------------------------- rescore + Top-k select
 constexpr int RS_NT = 256;
+constexpr int RS_GB = 4;  // groups of 16 candidates whose loads a warp keeps in flight
 
 
 
-template <int KPT>
+constexpr int RS_KPT = 4;                 // candidates per thread
+constexpr int RS_EPC = RS_NT * RS_KPT;    // candidates per CTA
+
 struct RescoreSmem {
-  SelectSmem<RS_NT> sel;
-  uint32_t keys[RS_NT * KPT];
-  int32_t blocks[RS_NT * KPT / CSA2_BLK];
+  SelectSmem<RS_NT, RS_KPT> sel;
+  alignas(16) uint32_t keys[RS_EPC];
+  int32_t blocks[RS_EPC / CSA2_BLK];
 };
 
 __device__ __forceinline__ int64_t pos_row(const RescoreParams& p, int b, int pos) {
@@ -255,11 +270,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int KPT>
 __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescoreParams p) {
-  constexpr int EPC = RS_NT * KPT;  // candidates per CTA
+  constexpr int EPC = RS_EPC;  // candidates per CTA
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  RescoreSmem<KPT>& s = *reinterpret_cast<RescoreSmem<KPT>*>(smem_raw);
+  RescoreSmem& s = *reinterpret_cast<RescoreSmem*>(smem_raw);
+  pdl_launch_dependents();
+  pdl_wait();  // the candidate blocks come from the previous kernel
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int b = blockIdx.y;
@@ -293,64 +309,78 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
   const float w0 = __ldg(job.w + b * CSA2_HI + 2 * c), w1 = __ldg(job.w + b * CSA2_HI + 2 * c + 1);
   __syncthreads();
 
-  // Score 16 candidates per warp step: rows grp and grp + 8 of the group.
-  for (int g = warp; g < EPC / 16; g += RS_NT / 32) {
-    uint32_t av[2][8];
-    bool valid[2];
+  // Score 16 candidates per MMA: rows grp and grp + 8 of a group.  A warp
+  // issues the row loads of RS_GB groups before their MMAs, so that several
+  // gathered rows are in flight per lane.
+  constexpr int NW = RS_NT / 32;
+  constexpr int GPW = EPC / 16 / NW;  // groups per warp
+  constexpr int GB = GPW < RS_GB ? GPW : RS_GB;
+  for (int gb = 0; gb < GPW; gb += GB) {
+    uint32_t av[GB][2][8];
+    bool valid[GB][2];
 #pragma unroll
-    for (int h = 0; h < 2; h++) {
-      const int e = g * 16 + grp + 8 * h;  // candidate index within this CTA
-      const int blk = s.blocks[e / CSA2_BLK];
-      const int pos = blk * CSA2_BLK + (e % CSA2_BLK);
-      int64_t row = -1;
-      valid[h] = blk >= 0 && pos < C;
-      if (valid[h]) {
-        row = pos_row(p, b, pos);
-        if (row < 0) {
-          set_status(p.status, ST_DEVICE_CHECK);
-          valid[h] = false;
+    for (int u = 0; u < GB; u++) {
+      const int g = warp + NW * (gb + u);
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int e = g * 16 + grp + 8 * h;  // candidate index within this CTA
+        const int blk = s.blocks[e / CSA2_BLK];
+        const int pos = blk * CSA2_BLK + (e % CSA2_BLK);
+        int64_t row = -1;
+        valid[u][h] = blk >= 0 && pos < C;
+        if (valid[u][h]) {
+          row = pos_row(p, b, pos);
+          if (row < 0) {
+            set_status(p.status, ST_DEVICE_CHECK);
+            valid[u][h] = false;
+          }
+        }
+        if (row >= 0) {
+          const uint4* kp = reinterpret_cast<const uint4*>(p.idx_k + row * CSA2_DI + 16 * c);
+          const uint4 k0 = __ldg(kp), k1 = __ldg(kp + 1);
+          av[u][h][0] = k0.x; av[u][h][1] = k0.y; av[u][h][2] = k0.z; av[u][h][3] = k0.w;
+          av[u][h][4] = k1.x; av[u][h][5] = k1.y; av[u][h][6] = k1.z; av[u][h][7] = k1.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; i++) av[u][h][i] = 0u;
         }
       }
-      if (row >= 0) {
-        const uint4* kp = reinterpret_cast<const uint4*>(p.idx_k + row * CSA2_DI + 16 * c);
-        const uint4 k0 = __ldg(kp), k1 = __ldg(kp + 1);
-        av[h][0] = k0.x; av[h][1] = k0.y; av[h][2] = k0.z; av[h][3] = k0.w;
-        av[h][4] = k1.x; av[h][5] = k1.y; av[h][6] = k1.z; av[h][7] = k1.w;
-      } else {
+    }
 #pragma unroll
-        for (int i = 0; i < 8; i++) av[h][i] = 0u;
+    for (int u = 0; u < GB; u++) {
+      const int g = warp + NW * (gb + u);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 4; ks++) {
+        const uint32_t a[4] = {av[u][0][2 * ks], av[u][1][2 * ks], av[u][0][2 * ks + 1],
+                               av[u][1][2 * ks + 1]};
+        mma_bf16_16816(d, a, bq[2 * ks], bq[2 * ks + 1]);
       }
-    }
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 4; ks++) {
-      const uint32_t a[4] = {av[0][2 * ks], av[1][2 * ks], av[0][2 * ks + 1], av[1][2 * ks + 1]};
-      mma_bf16_16816(d, a, bq[2 * ks], bq[2 * ks + 1]);
-    }
-    float s0 = fmaf(w1, fmaxf(d[1], 0.f), w0 * fmaxf(d[0], 0.f));
-    float s1 = fmaf(w1, fmaxf(d[3], 0.f), w0 * fmaxf(d[2], 0.f));
-    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-    if (c == 0) {
-      s.keys[g * 16 + grp] = valid[0] ? float_key(s0) : 0u;
-      s.keys[g * 16 + grp + 8] = valid[1] ? float_key(s1) : 0u;
+      float s0 = fmaf(w1, fmaxf(d[1], 0.f), w0 * fmaxf(d[0], 0.f));
+      float s1 = fmaf(w1, fmaxf(d[3], 0.f), w0 * fmaxf(d[2], 0.f));
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+      if (c == 0) {
+        s.keys[g * 16 + grp] = valid[u][0] ? float_key(s0) : 0u;
+        s.keys[g * 16 + grp + 8] = valid[u][1] ? float_key(s1) : 0u;
+      }
     }
   }
   __syncthreads();
 
-  uint32_t key[KPT];
-  int32_t id[KPT];
+  uint32_t key[RS_KPT];
 #pragma unroll
-  for (int j = 0; j < KPT; j++) {
-    const int e = t * KPT + j;
-    key[j] = s.keys[e];
-    const int blk = s.blocks[e / CSA2_BLK];
-    id[j] = blk * CSA2_BLK + (e % CSA2_BLK);
-  }
-  cluster_select_topk<RS_NT, KPT>(s.sel, key, id, p.top_k,
-                                  job.idx + (int64_t)b * job.idx_stride, job.idx_count + b);
+  for (int j = 0; j < RS_KPT; j++) key[j] = s.keys[t * RS_KPT + j];
+  const int32_t* blocks = s.blocks;
+  auto id_of = [blocks, e0](int e) {  // candidate index -> position
+    const int el = e - e0;
+    return blocks[el / CSA2_BLK] * CSA2_BLK + (el % CSA2_BLK);
+  };
+  __syncthreads();
+  cluster_select_topk<RS_NT, RS_KPT>(s.sel, key, id_of, p.top_k,
+                                     job.idx + (int64_t)b * job.idx_stride, job.idx_count + b);
 }
 
 // --------------------------------------------- block Top-k (pool) select
@@ -361,7 +391,10 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
     const float* __restrict__ bm, int32_t bm_stride, const int32_t* __restrict__ n_rows,
     int32_t max_rows, int32_t k_req, int32_t* sel, int32_t sel_stride, int32_t* sel_count,
     uint32_t* status) {
-  __shared__ SelectSmem<BS_NT> sm;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SelectSmem<BS_NT, BS_KPT>& sm = *reinterpret_cast<SelectSmem<BS_NT, BS_KPT>*>(smem_raw);
+  pdl_launch_dependents();
+  pdl_wait();  // the block maxima come from the scan
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int b = blockIdx.y;
@@ -369,7 +402,6 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
   const int nblk = (C + CSA2_BLK - 1) / CSA2_BLK;
   const int e0 = (rank * BS_NT + threadIdx.x) * BS_KPT;
   uint32_t key[BS_KPT];
-  int32_t id[BS_KPT];
   const float* src = bm + (int64_t)b * bm_stride + e0;
 #pragma unroll
   for (int j = 0; j < BS_KPT; j += 4) {
@@ -377,13 +409,10 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
     if (e0 + j < nblk) v = *reinterpret_cast<const float4*>(src + j);
     const float f[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int u = 0; u < 4; u++) {
-      key[j + u] = (e0 + j + u < nblk) ? float_key(f[u]) : 0u;
-      id[j + u] = e0 + j + u;
-    }
+    for (int u = 0; u < 4; u++) key[j + u] = (e0 + j + u < nblk) ? float_key(f[u]) : 0u;
   }
-  cluster_select_topk<BS_NT, BS_KPT>(sm, key, id, k_req, sel + (int64_t)b * sel_stride,
-                                     sel_count + b);
+  cluster_select_topk<BS_NT, BS_KPT>(sm, key, [](int e) { return e; }, k_req,
+                                     sel + (int64_t)b * sel_stride, sel_count + b);
 }
 
 // ------------------------------------------------------------ launchers
@@ -403,50 +432,40 @@ cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, cons
   return cudaGetLastError();
 }
 
-template <int KPT>
-static cudaError_t launch_rescore_t(const RescoreParams& p, int n_jobs, int batch, int cs,
-                                    cudaStream_t st) {
-  auto kern = rescore_select_kernel<KPT>;
-  const size_t smem = sizeof(RescoreSmem<KPT>);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  if (cs > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+// Candidates per sequence: n_cand_blocks * 8, RS_EPC per CTA of a cluster of
+// up to 16 CTAs that scores and selects them together.
+cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
+                           cudaStream_t st) {
+  const int ncand = n_cand_blocks * CSA2_BLK;
+  int cs = 1;
+  while (cs * RS_EPC < ncand) cs <<= 1;
+  if (cs > 16) return cudaErrorInvalidValue;
+  static bool attr_done = false;
+  const size_t smem = sizeof(RescoreSmem);
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(rescore_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(rescore_select_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, batch, n_jobs);
   cfg.blockDim = dim3(RS_NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = cs;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
-}
-
-// Candidates per sequence: n_cand_blocks * 8.  Picks a cluster of up to 16
-// CTAs of 256 threads holding 4 (else 16) candidates per thread.
-cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
-                           cudaStream_t st) {
-  const int ncand = n_cand_blocks * CSA2_BLK;
-  int cs = (ncand + RS_NT * 4 - 1) / (RS_NT * 4);
-  if (cs < 1) cs = 1;
-  if (cs <= 16) {
-    int c2 = 1;
-    while (c2 < cs) c2 <<= 1;
-    return launch_rescore_t<4>(p, n_jobs, batch, c2, st);
-  }
-  cs = (ncand + RS_NT * 16 - 1) / (RS_NT * 16);
-  int c2 = 1;
-  while (c2 < cs) c2 <<= 1;
-  if (c2 > 16) return cudaErrorInvalidValue;
-  return launch_rescore_t<16>(p, n_jobs, batch, c2, st);
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, rescore_select_kernel, p);
 }
 
 cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n_rows,
@@ -458,18 +477,28 @@ cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n
   int c2 = 1;
   while (c2 < cs) c2 <<= 1;
   if (c2 > 8) return cudaErrorInvalidValue;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(block_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(SelectSmem<BS_NT, BS_KPT>));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(c2, batch, 1);
   cfg.blockDim = dim3(BS_NT);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = sizeof(SelectSmem<BS_NT, BS_KPT>);
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = c2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, block_select_kernel, bm, (int32_t)bm_stride, n_rows,
                             (int32_t)max_rows, (int32_t)k_req, sel, (int32_t)sel_stride,
                             sel_count, status);

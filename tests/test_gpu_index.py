@@ -65,6 +65,45 @@ def test_index_full_parity(lib, orc, n_rows, pool_blocks, paged):
     check_full(orc, dw, 0, 512, pool_blocks, *out)
 
 
+@pytest.mark.parametrize("pool_blocks", [2048, 0])
+def test_index_full_exact_ties(lib, orc, pool_blocks):
+    """Indexer K rows repeat with period 37, so scores and block maxima tie
+    exactly (on both sides); the selection must follow the tie rule exactly:
+    lower position, lower block id."""
+    n_rows = [20000, 3000]
+    wl = synth.make("ties", seed=31, B=2, n_rows=n_rows, modes=[FULL], pool_blocks=pool_blocks)
+    dw = DeviceWorkload(lib, wl, orc)
+    k = dw.idxk_np.copy()
+    for b in range(wl.B):
+        base = b * wl.seq_stride
+        k[base:base + wl.seq_stride] = k[base + np.arange(wl.seq_stride) % 37]
+    dw.idxk_np = k
+    dw.idxk.copy_(dev(k))
+    idx, cnt, pool, pcnt = run_full(lib, dw, 0, 512, pool_blocks)
+    kv = dw.oracle_kv(orc)
+    for b in range(wl.B):
+        s = orc.scores(kv, orc.dims(), b, n_rows[b], wl.q_idx[0, b], wl.w_h[0, b])
+        assert np.array_equal(idx[b, :cnt[b]], orc.select_topk(s, 512)), b
+        if pool_blocks:
+            assert np.array_equal(pool[b, :pcnt[b]], orc.pool(orc.block_max(s, 8), pool_blocks))
+
+
+@pytest.mark.parametrize("pool_blocks", [2048, 0])
+def test_index_full_all_scores_equal(lib, orc, pool_blocks):
+    """A zero indexer query makes every score 0: the whole range ties, so the
+    first positions and the first blocks are selected."""
+    n_rows = [40000, 700]
+    wl = synth.make("zero", seed=32, B=2, n_rows=n_rows, modes=[FULL], pool_blocks=pool_blocks)
+    dw = DeviceWorkload(lib, wl, orc)
+    dw.q_idx.zero_()
+    idx, cnt, pool, pcnt = run_full(lib, dw, 0, 512, pool_blocks)
+    for b in range(wl.B):
+        assert np.array_equal(idx[b, :cnt[b]], np.arange(min(512, n_rows[b]))), b
+        if pool_blocks:
+            nb = (n_rows[b] + 7) // 8
+            assert np.array_equal(pool[b, :pcnt[b]], np.arange(min(pool_blocks, nb))), b
+
+
 def test_index_full_small_topk_and_pool(lib, orc):
     wl = synth.make("idx", seed=7, B=2, n_rows=[1234, 4321], modes=[FULL], pool_blocks=40)
     dw = DeviceWorkload(lib, wl, orc)
