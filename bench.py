@@ -283,7 +283,7 @@ def run_gpu(args, wl, rank, world):
     t_step = max_over_ranks(sum(times) / K, dist, dev)
 
     # ---- traced pass: per-launch events for the stage breakdown and roofline
-    n_ev = 16
+    n_ev = 32
     tev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev * K)]
     for e in tev:
         e.record(stream)

@@ -13,17 +13,16 @@
 // swizzled shared tile (E2M1 x E4M3 and E4M3 are exact in fp16), computes
 // S = Q K^T and O += P V with m16n8k16 tensor-core tiles (M = the 16 heads:
 // a per-step tile far too small for tcgen05's 64/128-row MMA), keeps the
-// online-softmax state in fp32.  The CTAs of one (layer, sequence) form a
-// thread-block cluster: at the end each publishes its unnormalised O, max and
-// sum in shared memory and the cluster merges them through distributed
-// shared memory (log-sum-exp weights), each CTA finishing a slice of the
-// output.  No partial result goes to HBM and no second kernel runs.
+// online-softmax state in fp32.  With one split the CTA normalises and writes
+// the output; otherwise each split writes its unnormalised O, max and sum
+// (coalesced, to the workspace, where they stay in L2) and attn_merge_kernel,
+// one CTA per (layer, sequence, head), combines them with log-sum-exp
+// weights.  Each thread derives its gather addresses from the indices
+// directly, and the query load overlaps the first gather.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
-
-#include <cooperative_groups.h>
 
 #include "csa2_internal.cuh"
 #include "kernels.h"
@@ -43,9 +42,6 @@ struct AttnSmem {
   __half p[CSA2_H * AT_CH];    // swizzled rows of 128 B
   float s[CSA2_H][AT_CH + 4];
   float m[CSA2_H], l[CSA2_H], alpha[CSA2_H];
-  float mall[16][CSA2_H], lall[16][CSA2_H];  // split merge: every rank's max and sum
-  float fr[16][CSA2_H];                      // weight of each rank's partial
-  float invl[CSA2_H];
   int64_t row[AT_CH];
 };
 
@@ -95,6 +91,7 @@ __device__ __forceinline__ int64_t kv_row(const AttnParams& p, int b, int pos) {
 __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   AttnSmem& s = *reinterpret_cast<AttnSmem*>(smem_raw);
+  pdl_launch_dependents();
   pdl_wait();  // the indices come from the previous kernel
   const int split = blockIdx.x, b = blockIdx.y, li = blockIdx.z;
   const AttnLayer L = p.layer[li];
@@ -168,11 +165,11 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
     const int nk = sparse ? n_idx : n_swa;
     if (k0 >= nk) continue;  // uniform across the CTA
     __syncthreads();         // previous chunk fully consumed
-    if (t < AT_CH) {
+    if (t < AT_CH) {  // validity of each key, for the logits mask
       int64_t row = -1;
       if (k0 + t < nk) {
         if (sparse) {
-          const int pos = idx[k0 + t];
+          const int pos = __ldg(idx + k0 + t);
           if (pos >= 0 && pos < C) row = kv_row(p, b, pos);
           if (row < 0) set_status(p.status, ST_DEVICE_CHECK);
         } else {
@@ -181,15 +178,19 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
       }
       s.row[t] = row;
     }
-    __syncthreads();
     if (sparse) {
-      // 64 rows x 16 chunks of 16 code bytes (32 channels, 2 scale groups).
+      // 64 rows x 16 chunks of 16 code bytes (32 channels, 2 scale groups);
+      // each thread resolves its own rows from the indices.
       uint4 cv[8];
       uint32_t sv[8];
 #pragma unroll
       for (int u = 0; u < 8; u++) {
         const int i = t + u * AT_NT, r = i >> 4, cc = i & 15;
-        const int64_t row = s.row[r];
+        int64_t row = -1;
+        if (k0 + r < nk) {
+          const int pos = __ldg(idx + k0 + r);
+          if (pos >= 0 && pos < C) row = kv_row(p, b, pos);
+        }
         if (row >= 0) {
           cv[u] = __ldg(reinterpret_cast<const uint4*>(p.codes + row * (CSA2_D / 2)) + cc);
           sv[u] = __ldg(reinterpret_cast<const uint16_t*>(p.scales + row * (CSA2_D / 16)) + cc);
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
 #pragma unroll
       for (int u = 0; u < 16; u++) {
         const int i = t + u * AT_NT, r = i >> 5, cc = i & 31;
-        const int64_t row = s.row[r];
+        const int64_t row = k0 + r < nk ? (int64_t)(k0 + r) : -1;
         cv[u] = row >= 0 ? __ldg(reinterpret_cast<const uint4*>(swa + row * CSA2_D) + cc)
                          : make_uint4(0, 0, 0, 0);
       }
@@ -365,63 +366,69 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
     }
     return;
   }
-  // Split merge across the cluster, push-only: after every rank has finished
-  // with its key/value tile, each rank writes its (max, sum) to every rank and
-  // each pair of its unnormalised O to the rank that owns that pair of output
-  // elements (into the owner's idle key/value tile); after a second cluster
-  // barrier every rank reduces its own slice from local shared memory.
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int ns = p.nsplit;
-  const int rank = (int)cluster.block_rank();
-  constexpr int NPAIR = CSA2_H * CSA2_D / 2;
-  const int slice = (NPAIR + ns - 1) / ns + 1;  // receive row length in pairs
-  cluster.sync();  // every rank is done with its key/value tile
-  if (t < CSA2_H) {
-    for (int r = 0; r < ns; r++) {
-      *cluster.map_shared_rank(&s.mall[rank][t], r) = s.m[t];
-      *cluster.map_shared_rank(&s.lall[rank][t], r) = s.l[t];
-    }
-  }
+  // Split partial: unnormalised O through the idle key/value tile (rows padded
+  // to 520 floats against bank conflicts) to coalesced 16-byte stores.
+  constexpr int OS = 520;
+  float* ob = reinterpret_cast<float*>(s.kv);
 #pragma unroll
   for (int nt = 0; nt < 16; nt++) {
-#pragma unroll
-    for (int hh = 0; hh < 2; hh++) {
-      const int row = g + 8 * hh;
-      const int q = (row * CSA2_D + warp * 128 + nt * 8 + 2 * tig) >> 1;  // pair index
-      const int owner = ((q + 1) * ns - 1) / NPAIR;
-      const int q0 = owner * NPAIR / ns;
-      float2* dst = reinterpret_cast<float2*>(s.kv) + rank * slice + (q - q0);
-      *cluster.map_shared_rank(dst, owner) = make_float2(o[nt][2 * hh], o[nt][2 * hh + 1]);
-    }
-  }
-  cluster.sync();  // all pushes have landed; no remote access after this
-  if (t < CSA2_H) {
-    float mx = -INFINITY;
-    for (int r = 0; r < ns; r++) mx = fmaxf(mx, s.mall[r][t]);
-    float den = 0.f;
-    for (int r = 0; r < ns; r++) {
-      const float mr = s.mall[r][t];
-      const float f = (mx == -INFINITY || mr == -INFINITY) ? 0.f : exp2f(mr - mx);
-      s.fr[r][t] = f;
-      den += f * s.lall[r][t];
-    }
-    s.invl[t] = den > 0.f ? 1.0f / den : 0.f;
+    const int ch = warp * 128 + nt * 8 + 2 * tig;
+    *reinterpret_cast<float2*>(ob + g * OS + ch) = make_float2(o[nt][0], o[nt][1]);
+    *reinterpret_cast<float2*>(ob + (g + 8) * OS + ch) = make_float2(o[nt][2], o[nt][3]);
   }
   __syncthreads();
-  const int q0 = rank * NPAIR / ns, q1 = (rank + 1) * NPAIR / ns;
-  const float2* recv = reinterpret_cast<const float2*>(s.kv);
-  for (int q = q0 + t; q < q1; q += AT_NT) {
-    const int h = (2 * q) / CSA2_D;
-    float a0 = 0.f, a1 = 0.f;
-    for (int r = 0; r < ns; r++) {
-      const float2 v = recv[r * slice + (q - q0)];
-      a0 = fmaf(s.fr[r][h], v.x, a0);
-      a1 = fmaf(s.fr[r][h], v.y, a1);
-    }
-    *reinterpret_cast<__nv_bfloat162*>(out + 2 * q) =
-        __floats2bfloat162_rn(a0 * s.invl[h], a1 * s.invl[h]);
+  const int64_t slot = ((int64_t)li * p.batch + b) * p.nsplit + split;
+  float4* dst = reinterpret_cast<float4*>(p.part_o + slot * (CSA2_H * CSA2_D));
+  for (int i = t; i < CSA2_H * CSA2_D / 4; i += AT_NT) {
+    const int row = i >> 7, c4 = i & 127;
+    dst[i] = *reinterpret_cast<const float4*>(ob + row * OS + 4 * c4);
   }
+  if (t < CSA2_H)
+    *reinterpret_cast<float2*>(p.part_ml + (slot * CSA2_H + t) * 2) = make_float2(s.m[t], s.l[t]);
+}
+
+// Log-sum-exp merge of the split partials of one (layer, sequence, head).
+__global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
+  pdl_wait();  // the partials come from attn_decode_kernel
+  const int h = blockIdx.x, b = blockIdx.y, li = blockIdx.z;
+  const int t = threadIdx.x, ns = p.nsplit;
+  const int64_t slot0 = ((int64_t)li * p.batch + b) * ns;
+  __shared__ float f[16];
+  __shared__ float invl;
+  if (t < 32) {
+    float m = -INFINITY, l = 0.f;
+    if (t < ns) {
+      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + ((slot0 + t) * CSA2_H + h) * 2);
+      m = ml.x;
+      l = ml.y;
+    }
+    float mx = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float fw = (mx == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - mx);
+    float den = fw * l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (t < ns) f[t] = fw;
+    if (t == 0) invl = den > 0.f ? 1.0f / den : 0.f;
+  }
+  __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < ns; r++) {
+    const float4 v = *reinterpret_cast<const float4*>(p.part_o + (slot0 + r) * (CSA2_H * CSA2_D) +
+                                                      h * CSA2_D + 4 * t);
+    acc.x = fmaf(f[r], v.x, acc.x);
+    acc.y = fmaf(f[r], v.y, acc.y);
+    acc.z = fmaf(f[r], v.z, acc.z);
+    acc.w = fmaf(f[r], v.w, acc.w);
+  }
+  uint16_t* out = p.layer[li].out + ((int64_t)b * CSA2_H + h) * CSA2_D + 4 * t;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * invl, acc.y * invl);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * invl, acc.w * invl);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(out) = pk;
 }
 
 int attn_nsplit(int pairs, int num_sms) {
@@ -438,27 +445,35 @@ cudaError_t launch_attn(const AttnParams& p, cudaStream_t st) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(AttnSmem));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  trace_mark("attn", st);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.nsplit, p.batch, p.n_layers);
   cfg.blockDim = dim3(AT_NT);
   cfg.dynamicSmemBytes = sizeof(AttnSmem);
   cfg.stream = st;
-  cudaLaunchAttribute at[2];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = p.nsplit;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, attn_decode_kernel, p);
+  cfg.numAttrs = 1;
+  trace_mark("attn", st);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_decode_kernel, p);
+  if (e != cudaSuccess || p.nsplit == 1) return e;
+  cudaLaunchConfig_t mc = {};
+  mc.gridDim = dim3(CSA2_H, p.batch, p.n_layers);
+  mc.blockDim = dim3(128);
+  mc.stream = st;
+  mc.attrs = at;
+  mc.numAttrs = 1;
+  trace_mark("attn_merge", st);
+  return cudaLaunchKernelEx(&mc, attn_merge_kernel, p);
 }
 
+size_t attn_partial_bytes(int batch, int n_layers, int nsplit) {
+  if (nsplit <= 1) return 0;
+  const size_t slots = (size_t)batch * n_layers * nsplit;
+  return slots * CSA2_H * CSA2_D * sizeof(float) + slots * CSA2_H * 2 * sizeof(float);
+}
 
 }  // namespace csa2

@@ -191,6 +191,8 @@ static int cand_blocks_max(const csa2_kv_view* kv, int P) {
 // ------------------------------------------------------------ group plan
 struct GroupWs {
   IndexWs ix;
+  float* part_o;
+  float* part_ml;
   int nsplit;
   size_t bytes;
 };
@@ -199,7 +201,10 @@ static GroupWs group_ws_layout(const csa2_group_desc* d, uint8_t* base) {
   GroupWs g{};
   g.ix = index_ws_layout(&d->kv, d->top_k, base);
   g.nsplit = attn_nsplit(d->kv.batch * d->n_layers, num_sms());
-  g.bytes = g.ix.bytes;
+  const size_t slots = (size_t)d->kv.batch * d->n_layers * g.nsplit;
+  g.part_o = reinterpret_cast<float*>(base + g.ix.bytes);
+  g.part_ml = reinterpret_cast<float*>(base + g.ix.bytes + slots * CSA2_H * CSA2_D * sizeof(float));
+  g.bytes = g.ix.bytes + align256(attn_partial_bytes(d->kv.batch, d->n_layers, g.nsplit));
   return g;
 }
 
@@ -288,7 +293,8 @@ csa2_status csa2_index_reindex(const csa2_kv_view* kv, const uint16_t* q_idx, co
 
 size_t csa2_attn_workspace_size(int32_t batch, int32_t n_layers) {
   if (batch < 1 || n_layers < 1) return 0;
-  return CSA2_WS_HEADER;  // the status word only
+  const int ns = attn_nsplit(batch * n_layers, num_sms());
+  return CSA2_WS_HEADER + align256(attn_partial_bytes(batch, n_layers, ns));
 }
 
 static csa2_status fill_attn_common(AttnParams& ap, const csa2_kv_view* kv, const int32_t* swa_len,
@@ -332,6 +338,10 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, const csa2_kv_view* kv, c
   ap.n_layers = 1;
   ap.nsplit = attn_nsplit(kv->batch, num_sms());
   ap.layer[0] = AttnLayer{q, swa, idx, idx_count, nullptr, nullptr, out};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t slots = (size_t)kv->batch * ap.nsplit;
+  ap.part_o = reinterpret_cast<float*>(base + CSA2_WS_HEADER);
+  ap.part_ml = reinterpret_cast<float*>(base + CSA2_WS_HEADER + slots * CSA2_H * CSA2_D * 4);
   ap.status = static_cast<uint32_t*>(ws);
   CSA2_CUDA(launch_attn(ap, (cudaStream_t)stream));
   trace_mark("end", (cudaStream_t)stream);
@@ -419,6 +429,8 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
   fill_attn_common(ap, kv, d->swa_len, d->sm_scale, K);
   ap.n_layers = L;
   ap.nsplit = g.nsplit;
+  ap.part_o = g.part_o;
+  ap.part_ml = g.part_ml;
   ap.status = g.ix.status;
   int src = 0;
   for (int l = 0; l < L; l++) {

@@ -84,9 +84,12 @@ struct AttnParams {
   const int32_t* n_rows;
   const int32_t* swa_len;
   float scale_log2;
+  float* part_o;   // [n_layers][batch][nsplit][16][512] split partials (nsplit > 1)
+  float* part_ml;  // [n_layers][batch][nsplit][16][2] their max and sum
   uint32_t* status;
 };
 int attn_nsplit(int pairs, int num_sms);
+size_t attn_partial_bytes(int batch, int n_layers, int nsplit);
 cudaError_t launch_attn(const AttnParams& p, cudaStream_t st);
 
 }  // namespace csa2
