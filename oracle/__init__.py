@@ -90,6 +90,12 @@ def lib():
                                         C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
                                         C.c_int32, C.c_double, C.c_void_p, C.c_void_p,
                                         C.c_void_p, C.c_void_p, C.c_void_p]
+        L.csa2o_project_idxk.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
+                                         C.c_void_p]
+        L.csa2o_cache_append.argtypes = [C.POINTER(_KV), C.POINTER(_Dims), C.c_int32,
+                                         C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                         C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p,
+                                         C.c_void_p, C.c_void_p, C.c_void_p]
     return _lib
 
 
@@ -251,3 +257,38 @@ def layer_group(kv: KV, dm, n_rows, modes, q_idx, w, q, swa, swa_len, *, top_k=5
         raise ValueError("oracle layer group: bad arguments or row outside the pool")
     return dict(idx=idx, idx_count=idx_count, pool=pool_[:, :pool_blocks],
                 pool_count=pool_count, out=out)
+
+
+# ---------------------------------------------------- cache append (next row)
+def project_idxk(x_bf16: np.ndarray, w_idx: np.ndarray) -> np.ndarray:
+    """bf16 indexer-K row of one bf16 main-KV entry (fp64 sum, bf16 RNE)."""
+    x = _c(x_bf16, np.uint16)
+    w = _c(w_idx, np.uint16)
+    d, di = w.shape
+    out = np.zeros(di, np.uint16)
+    if lib().csa2o_project_idxk(_p(x), _p(w), d, di, _p(out)):
+        raise ValueError("oracle project_idxk: bad arguments")
+    return out
+
+
+def cache_append(kv: KV, dm, n_rows: np.ndarray, x: np.ndarray, w_idx: np.ndarray,
+                 x_swa: np.ndarray | None = None, swa: np.ndarray | None = None,
+                 swa_pos: np.ndarray | None = None, swa_len: np.ndarray | None = None) -> int:
+    """Append one step's entries in place: kv.codes/scales/idxk rows, n_rows
+    (int64), and the window rings swa[L][B][w][d] with swa_pos (int64) and
+    swa_len (int32).  Returns the oracle's return code (1 when a sequence's
+    row is not mapped; that sequence is skipped)."""
+    B = len(n_rows)
+    for a, dt in ((n_rows, np.int64), (x, np.uint16), (w_idx, np.uint16)):
+        if a.dtype != dt or not a.flags.c_contiguous:
+            raise TypeError("cache_append: arrays must be C-contiguous of the documented dtype")
+    L = 0 if x_swa is None else x_swa.shape[0]
+    if L:
+        for a, dt in ((x_swa, np.uint16), (swa, np.uint8), (swa_pos, np.int64),
+                      (swa_len, np.int32)):
+            if a.dtype != dt or not a.flags.c_contiguous:
+                raise TypeError("cache_append: arrays must be C-contiguous of the documented dtype")
+    return lib().csa2o_cache_append(C.byref(kv.s), C.byref(dm), B, _p(kv.codes), _p(kv.scales),
+                                    _p(kv.idxk), _p(n_rows), _p(x), _p(w_idx), L,
+                                    _p(x_swa) if L else None, _p(swa) if L else None,
+                                    _p(swa_pos) if L else None, _p(swa_len) if L else None)

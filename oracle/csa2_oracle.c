@@ -375,3 +375,51 @@ int csa2o_layer_group(const csa2o_kv *kv, const csa2o_dims *dm, int32_t B,
   }
   return rc;
 }
+
+/* ----------------------------------------------------------- cache append */
+
+int csa2o_project_idxk(const uint16_t *x, const uint16_t *w_idx, int32_t d, int32_t di,
+                       uint16_t *out) {
+  if (d <= 0 || di <= 0) return CSA2O_EARG;
+  for (int32_t j = 0; j < di; j++) {
+    double acc = 0.0;
+    for (int32_t c = 0; c < d; c++)
+      acc += csa2o_bf16_value(x[c]) * csa2o_bf16_value(w_idx[(int64_t)c * di + j]);
+    out[j] = csa2o_bf16_round(acc);
+  }
+  return CSA2O_OK;
+}
+
+int csa2o_cache_append(const csa2o_kv *kv, const csa2o_dims *dm, int32_t B,
+                       uint8_t *codes, uint8_t *scales, uint16_t *idxk,
+                       int64_t *n_rows, const uint16_t *x, const uint16_t *w_idx,
+                       int32_t L, const uint16_t *x_swa, uint8_t *swa,
+                       int64_t *swa_pos, int32_t *swa_len) {
+  const int32_t d = dm->d, di = dm->di, w = dm->w;
+  int rc = CSA2O_OK;
+  for (int32_t b = 0; b < B; b++) {
+    const int64_t p = n_rows[b];
+    const int64_t cap = kv->page_table ? (int64_t)kv->max_pages * kv->page_rows
+                                       : kv->seq_stride;
+    const int64_t row = (p >= 0 && p < cap) ? csa2o_row_of(kv, b, p) : -1;
+    if (row < 0) {
+      rc = CSA2O_EARG;
+      continue;
+    }
+    csa2o_quantize_fp4(x + (int64_t)b * d, 1, d, codes + row * (d / 2),
+                       scales + row * (d / 16));
+    csa2o_project_idxk(x + (int64_t)b * d, w_idx, d, di, idxk + row * di);
+    n_rows[b] = p + 1;
+  }
+  for (int32_t b = 0; b < B && L > 0; b++) {
+    const int64_t slot = swa_pos[b] % w;
+    for (int32_t l = 0; l < L; l++) {
+      const uint16_t *src = x_swa + ((int64_t)l * B + b) * d;
+      uint8_t *dst = swa + (((int64_t)l * B + b) * w + slot) * d;
+      for (int32_t c = 0; c < d; c++) dst[c] = csa2o_e4m3_encode((float)csa2o_bf16_value(src[c]));
+    }
+    swa_pos[b] += 1;
+    swa_len[b] = (int32_t)(swa_pos[b] < w ? swa_pos[b] : w);
+  }
+  return rc;
+}

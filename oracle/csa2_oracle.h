@@ -160,6 +160,40 @@ int csa2o_attention(const csa2o_kv *kv, const csa2o_dims *dm, int32_t b,
                     int32_t n_idx, const uint8_t *swa /*[w][d]*/,
                     int32_t swa_len, double sm_scale, double *out /*[h][d]*/);
 
+/* --------------------------------------- cache append (next row of work) */
+
+/* Indexer-K projection of one main-KV entry:
+ *   out[j] = bf16_RNE( sum_c x[c] * w_idx[c * di + j] ),  c < d, j < di
+ * with x and w_idx bf16, every product exact and the sum in fp64.  The
+ * pages say the indexer K is projected from the main KV entry instead of a
+ * separate compression of the hidden state [YOM §二 last paragraph; TUC
+ * §CSA2]; this build projects the entry as produced (bf16, before its FP4
+ * storage rounding) with a d x di bf16 matrix. */
+int csa2o_project_idxk(const uint16_t *x /*[d]*/, const uint16_t *w_idx /*[d][di]*/,
+                       int32_t d, int32_t di, uint16_t *out /*[di]*/);
+
+/* Append one decode step's new entries (one global entry per sequence, one
+ * sliding-window entry per layer and sequence):
+ *   for each b: p = n_rows[b]; row = csa2o_row_of(kv, b, p); the position must
+ *     also be below the sequence's capacity (seq_stride when contiguous,
+ *     max_pages * page_rows when paged);
+ *     codes/scales[row] = csa2o_quantize_fp4(x[b]) ; idxk[row] =
+ *     csa2o_project_idxk(x[b]) ; n_rows[b] = p + 1.
+ *     A sequence whose row is not mapped is left as it is (its counters too)
+ *     and the call returns CSA2O_EARG after processing the others.
+ *   for each layer l and b: slot = swa_pos[b] % w ;
+ *     swa[l][b][slot][c] = E4M3_RNE_satfinite(x_swa[l][b][c]) ;
+ *   then swa_pos[b] += 1, swa_len[b] = min(swa_pos[b], w).
+ * The main KV is FP4 with E4M3 scales and the window KV stays FP8 [YOM §三];
+ * each layer keeps its own window [REL §CSA2].  Storing the window entry
+ * without a scale, and as a ring of w slots, is this build's reading. */
+int csa2o_cache_append(const csa2o_kv *kv, const csa2o_dims *dm, int32_t B,
+                       uint8_t *codes, uint8_t *scales, uint16_t *idxk,
+                       int64_t *n_rows, const uint16_t *x /*[B][d]*/,
+                       const uint16_t *w_idx /*[d][di]*/, int32_t L,
+                       const uint16_t *x_swa /*[L][B][d]*/, uint8_t *swa /*[L][B][w][d]*/,
+                       int64_t *swa_pos /*[B]*/, int32_t *swa_len /*[B]*/);
+
 #ifdef __cplusplus
 }
 #endif
