@@ -5,7 +5,9 @@
 //    causally visible position; yomxxx.com CSA2 notes, section 二, HSI
 //    paragraph: it keeps the top 2,048 blocks of 8 positions by block max].
 //    It streams the bf16 indexer K (128 B per position) from HBM with TMA
-//    into a 5-stage shared-memory ring (128B-swizzled tiles of 128 positions),
+//    into a 3-stage shared-memory ring (128B-swizzled tiles of 128 positions),
+//    four CTAs per SM (four independent producer/MMA/epilogue pipelines keep
+//    more requests in flight than one deep ring per CTA does),
 //    one thread issues tcgen05.mma (M = 128 positions, N = 16 >= 8 indexer
 //    heads, K = 64) into a double-buffered TMEM accumulator, and four
 //    epilogue warps read the dot products back (tcgen05.ld), apply
@@ -27,7 +29,8 @@ namespace csa2 {
 // ------------------------------------------------------------- the scan
 constexpr int SC_BOX = 64;                 // rows per TMA box
 constexpr int SC_N = 16;                   // indexer heads padded to MMA N
-constexpr int SC_STAGES = 6;
+constexpr int SC_STAGES = 3;
+constexpr int SC_CTAS_PER_SM = 4;          // four independent pipelines per SM
 constexpr int SC_ACC = 4;                  // TMEM accumulator buffers (16 columns each)
 constexpr int SC_A_BYTES = SC_TILE * 128;  // 16 KB of indexer K per stage
 constexpr int SC_B_BYTES = SC_N * 128;     // 2 KB of indexer query per stage
@@ -74,7 +77,7 @@ __device__ __forceinline__ int32_t box_row(const ScanParams& p, int b, int pos0)
   return (int32_t)row;
 }
 
-__global__ void __launch_bounds__(SC_THREADS, 1)
+__global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
     score_scan_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_q, const ScanParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -426,7 +429,8 @@ cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, cons
     attr_done = true;
   }
   const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
-  const int grid = (int)(total < 2LL * num_sms ? total : 2LL * num_sms);
+  const int64_t slots = (int64_t)SC_CTAS_PER_SM * num_sms;
+  const int grid = (int)(total < slots ? total : slots);
   if (grid <= 0) return cudaSuccess;
   score_scan_kernel<<<grid, SC_THREADS, SC_SMEM, st>>>(map_k, map_q, p);
   return cudaGetLastError();

@@ -88,11 +88,13 @@ def test_index_full_exact_ties(lib, orc, pool_blocks):
             assert np.array_equal(pool[b, :pcnt[b]], orc.pool(orc.block_max(s, 8), pool_blocks))
 
 
-@pytest.mark.parametrize("pool_blocks", [2048, 0])
-def test_index_full_all_scores_equal(lib, orc, pool_blocks):
+@pytest.mark.parametrize("pool_blocks,n_rows", [(2048, [40000, 700]), (0, [40000, 700]),
+                                               (2048, [100000, 65])])
+def test_index_full_all_scores_equal(lib, orc, pool_blocks, n_rows):
     """A zero indexer query makes every score 0: the whole range ties, so the
-    first positions and the first blocks are selected."""
-    n_rows = [40000, 700]
+    first positions and the first blocks are selected.  At 100,000 rows the
+    tied block maxima outnumber what the bounded gather holds, so the block
+    selection takes its radix path."""
     wl = synth.make("zero", seed=32, B=2, n_rows=n_rows, modes=[FULL], pool_blocks=pool_blocks)
     dw = DeviceWorkload(lib, wl, orc)
     dw.q_idx.zero_()
