@@ -90,6 +90,8 @@ _index_reindex = _sig("csa2_index_reindex", C.c_int,
 _attn_ws = _sig("csa2_attn_workspace_size", _sz, [_i32, _i32])
 _attn = _sig("csa2_sparse_attn_decode", C.c_int,
              [_vp, C.POINTER(KVView), _vp, _vp, _i32, _vp, _vp, C.c_float, _vp, _vp, _sz, _vp])
+_append = _sig("csa2_cache_append", C.c_int,
+                [C.POINTER(KVView), _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _trace_set = _sig("csa2_trace_set", None, [_vp])
 _group_ws = _sig("csa2_group_workspace_size", _sz, [C.POINTER(GroupDesc)])
 _group = _sig("csa2_layer_group", C.c_int, [C.POINTER(GroupDesc), _vp, _sz, _vp])
@@ -202,6 +204,17 @@ def csa2_sparse_attn_decode(q, kv: KVCache, idx, idx_count, idx_stride, swa, swa
     _check(_attn(_ptr(q), C.byref(kv.view), _ptr(idx), _ptr(idx_count), idx_stride, _ptr(swa),
                  _ptr(swa_len), float(sm_scale), _ptr(out), _ptr(ws), ws.numel(),
                  _stream(stream)))
+
+
+def csa2_cache_append(kv: KVCache, x, w_idx, ws, x_swa=None, swa=None, swa_pos=None,
+                      swa_len=None, stream=None):
+    """Append one step's entries: x bf16 [B][512] into the FP4 cache and its
+    indexer K (w_idx bf16 [512][64]) at kv.n_rows (which advances), and
+    x_swa bf16 [L][B][512] into the E4M3 window rings swa [L][B][128][512] at
+    swa_pos % 128 (swa_pos advances, swa_len follows)."""
+    L = 0 if x_swa is None else int(x_swa.shape[0])
+    _check(_append(C.byref(kv.view), _ptr(x), _ptr(w_idx), L, _ptr(x_swa), _ptr(swa),
+                   _ptr(swa_pos), _ptr(swa_len), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 class LayerGroup:

@@ -208,6 +208,7 @@ static GroupWs group_ws_layout(const csa2_group_desc* d, uint8_t* base) {
   return g;
 }
 
+
 }  // namespace csa2
 
 using namespace csa2;
@@ -448,5 +449,49 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
   trace_mark("end", st);
   return CSA2_OK;
 }
+
+// ------------------------------------------------------------ cache append
+csa2_status csa2_cache_append(const csa2_kv_view* kv, const uint16_t* x, const uint16_t* w_idx,
+                              int32_t n_layers, const uint16_t* x_swa, uint8_t* swa,
+                              int32_t* swa_pos, int32_t* swa_len, void* ws, size_t ws_bytes,
+                              csa2_stream_t stream) {
+  csa2_status r = check_kv(kv);
+  if (r) return r;
+  CSA2_REQUIRE_PTR(x);
+  CSA2_REQUIRE_PTR(w_idx);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  CSA2_REQUIRE(n_layers >= 0 && n_layers <= 65535 * 4, CSA2_ERR_SHAPE, "n_layers = %d", n_layers);
+  if (n_layers > 0) {
+    CSA2_REQUIRE_PTR(x_swa);
+    CSA2_REQUIRE_PTR(swa);
+    CSA2_REQUIRE(swa_pos != nullptr && swa_len != nullptr, CSA2_ERR_INVALID_ARG,
+                 "swa_pos and swa_len are required when n_layers > 0");
+  }
+  AppendParams p{};
+  p.codes = const_cast<uint8_t*>(kv->codes);
+  p.scales = const_cast<uint8_t*>(kv->scales);
+  p.idx_k = const_cast<uint16_t*>(kv->idx_k);
+  p.page_table = kv->page_table;
+  p.max_pages = kv->max_pages;
+  p.seq_stride = kv->seq_stride;
+  p.pool_rows = kv->pool_rows;
+  p.n_rows = const_cast<int32_t*>(kv->n_rows);
+  p.batch = kv->batch;
+  p.x = x;
+  p.w_idx = w_idx;
+  p.n_layers = n_layers;
+  p.x_swa = x_swa;
+  p.swa = swa;
+  p.swa_pos = swa_pos;
+  p.swa_len = swa_len;
+  p.status = static_cast<uint32_t*>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  CSA2_CUDA(launch_append(p, st));
+  trace_mark("end", st);
+  return CSA2_OK;
+}
+
 
 }  // extern "C"

@@ -92,4 +92,26 @@ int attn_nsplit(int pairs, int num_sms);
 size_t attn_partial_bytes(int batch, int n_layers, int nsplit);
 cudaError_t launch_attn(const AttnParams& p, cudaStream_t st);
 
+// ------------------------------------------------------------ cache append
+struct AppendParams {
+  uint8_t* codes;
+  uint8_t* scales;
+  uint16_t* idx_k;
+  const int32_t* page_table;
+  int32_t max_pages;
+  int64_t seq_stride;
+  int64_t pool_rows;
+  int32_t* n_rows;
+  int32_t batch;
+  const uint16_t* x;       // [batch][512] new main-KV entries, bf16
+  const uint16_t* w_idx;   // [512][64] indexer-K projection, bf16
+  int32_t n_layers;
+  const uint16_t* x_swa;   // [n_layers][batch][512] new window entries, bf16
+  uint8_t* swa;            // [n_layers][batch][128][512] E4M3 window rings
+  int32_t* swa_pos;        // [batch] window entries written so far
+  int32_t* swa_len;        // [batch] valid window rows
+  uint32_t* status;
+};
+cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
+
 }  // namespace csa2

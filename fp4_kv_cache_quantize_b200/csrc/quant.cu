@@ -1,10 +1,6 @@
 // quant.cu -- FP4 main-KV pack (quantise) and unpack (dequantise) kernels.
 //
-// Format: E2M1 codes with one E4M3 scale per 16 channels and no global
-// scale, i.e. NVFP4 without its second-level scale (release note
-// "DeepSeek-V4.1-Flash 发布：100 万上下文 + FP4 KV Cache + 跨层注意力复用",
-// section "FP4 KV、Bounded Replay 及其他扩展"; yomxxx.com CSA2 paper notes,
-// section 三 "FP4 与部署侧的两个数字池").
+// Format: see fp4_codec.cuh.
 //
 // Both kernels are pure HBM streams: 16-byte coalesced loads and stores, a
 // grid of a few CTAs per SM looping over the data, no shared memory.
@@ -14,6 +10,7 @@
 #include <cuda_fp8.h>
 
 #include "csa2_internal.cuh"
+#include "fp4_codec.cuh"
 
 namespace csa2 {
 
@@ -23,22 +20,6 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// x / s for an E4M3 scale s, exact enough for E2M1 rounding: q0 = x * (1/s)
-// is refined with one fused residual step.  When x/s is exactly an E2M1
-// rounding midpoint (x = T*s, T in {.25,.75,1.25,1.75,2.5,3.5,5}) the result
-// is exactly T, so ties round as they would from the true quotient; every
-// other quotient of a bf16 by an E4M3 value lies at least ~2^-9 (relative)
-// away from every midpoint, far beyond the few-ulp error of q0.  The sign is
-// copied from x because the residual step turns x = -0 into +0.
-__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
-  const float q0 = __fmul_rn(x, r);
-  const float res = __fmaf_rn(-q0, s, x);
-  return copysignf(__fmaf_rn(res, r, q0), x);
 }
 
 // One thread packs one 16-byte chunk (8 channels); lanes 2j and 2j+1 share a
@@ -61,32 +42,15 @@ __global__ void __launch_bounds__(256) fp4_pack_kernel(const uint4* __restrict__
 #pragma unroll
     for (int u = 0; u < U; u++) {
       const int64_t i = base + u * stride;
-      float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
-                    bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
-      float amax = 0.0f;
-#pragma unroll
-      for (int k = 0; k < 8; k++) amax = fmaxf(amax, fabsf(f[k]));
+      float f[8];
+      unpack_bf16x8(v[u], f);
+      float amax = amax8(f);
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      // scale = E4M3(amax / 6): one correctly rounded fp32 division, then
-      // the hardware's round-to-nearest-even, saturate-to-finite conversion.
-      const float t = __fdiv_rn(amax, 6.0f);
-      const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3);
-      const float s = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
-      uint32_t packed = 0;
-      if (s != 0.0f) {
-        const float r = __frcp_rn(s);
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-          const float2 qq = make_float2(div_by_scale(f[2 * k], s, r),
-                                        div_by_scale(f[2 * k + 1], s, r));
-          const uint32_t byte =
-              (uint32_t)__nv_cvt_float2_to_fp4x2(qq, __NV_E2M1, cudaRoundNearest);
-          packed |= (byte & 0xFFu) << (8 * k);
-        }
-      }
+      uint8_t sb;
+      const uint32_t packed = fp4_encode8(f, amax, &sb);
       if (i < n_chunks) {
         codes[i] = packed;
-        if ((i & 1) == 0) scales[i >> 1] = (uint8_t)sb;
+        if ((i & 1) == 0) scales[i >> 1] = sb;
       }
     }
   }

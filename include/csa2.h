@@ -111,6 +111,44 @@ csa2_status csa2_workspace_init(void *ws, size_t ws_bytes, csa2_stream_t stream)
  * first device-side problem recorded since the last call. */
 csa2_status csa2_sync_status(void *ws, csa2_stream_t stream);
 
+/* --------------------------------------------------------- cache append */
+
+/*
+ * Append one decode step's new entries to the caches (the step that runs
+ * before csa2_layer_group; yomxxx.com CSA2 paper notes, section 二, last
+ * paragraph, and section 三; release note, section "Compressed Sparse
+ * Attention 2 (CSA2)"):
+ *   for each sequence b, at position p = kv->n_rows[b]:
+ *     codes/scales row of p  <- FP4 of x[b] (as csa2_quantize_fp4),
+ *     idx_k row of p         <- bf16_rne(x[b] @ w_idx)  (fp32 accumulation),
+ *     kv->n_rows[b]          <- p + 1;
+ *   for each layer l < n_layers and sequence b, at slot s = swa_pos[b] % 128:
+ *     swa[l][b][s][:]        <- E4M3 (round to nearest even, saturating to
+ *                               +-448, no scale) of x_swa[l][b][:],
+ *   then swa_pos[b] += 1 and swa_len[b] = min(swa_pos[b], 128).
+ * Arguments (device memory, caller-owned, 16-byte aligned):
+ *   kv      the cache; its codes, scales, idx_k and n_rows arrays are
+ *           WRITTEN by this call (the view's const qualifiers notwithstanding).
+ *           The new position must lie below the sequence's capacity
+ *           (seq_stride rows when contiguous, max_pages * 64 when paged) on a
+ *           mapped page; kv->max_rows is not checked against it (raise it
+ *           before the next decode step reads the longer sequence).
+ *   x       bf16 [batch][512]; w_idx bf16 [512][64];
+ *   n_layers >= 0 window layers; when 0, x_swa, swa, swa_pos and swa_len
+ *           may be NULL;  x_swa bf16 [n_layers][batch][512];
+ *           swa E4M3 [n_layers][batch][128][512];  swa_pos, swa_len int32
+ *           [batch], swa_pos >= 0.
+ *   ws      a workspace of at least CSA2_WS_HEADER bytes (status word).
+ * Errors: argument problems return before any launch.  A position with no
+ * row (full sequence, unmapped page) or a negative swa_pos leaves that
+ * sequence's cache and counters unchanged and records CSA2_ERR_DEVICE_CHECK
+ * for csa2_sync_status.  Two launches; asynchronous on stream.
+ */
+csa2_status csa2_cache_append(const csa2_kv_view *kv, const uint16_t *x, const uint16_t *w_idx,
+                              int32_t n_layers, const uint16_t *x_swa, uint8_t *swa,
+                              int32_t *swa_pos, int32_t *swa_len, void *ws, size_t ws_bytes,
+                              csa2_stream_t stream);
+
 /* ---------------------------------------------------------------- tracing */
 
 /*
