@@ -201,6 +201,51 @@ def config_dict(wl):
 
 
 # ------------------------------------------------------------ GPU arm
+def time_cache_append(csa2, wl, dev, stream, K, W):
+    """The cache-append step that precedes a decode step (one new main-KV
+    entry per sequence, one window entry per layer and sequence), timed with
+    events over K back-to-back calls into a scratch cache of the workload's
+    batch and layer count.  Latency-bound: it moves ~100 KB per call."""
+    import torch
+    B, L = wl.B, wl.L
+    cap = 64 * ((W + K + 63) // 64 + 1)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed)
+    codes = torch.zeros((B * cap, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B * cap, 32), dtype=torch.uint8, device=dev)
+    idxk = torch.zeros((B * cap, 64), dtype=torch.int16, device=dev)
+    n_rows = torch.zeros(B, dtype=torch.int32, device=dev)
+    kv = csa2.KVCache(codes, scales, idxk, n_rows, max_rows=cap, seq_stride=cap)
+    x = torch.randn((B, 512), generator=g, device=dev).to(torch.bfloat16).view(torch.int16)
+    w_idx = (torch.randn((512, 64), generator=g, device=dev) / 512 ** 0.5).to(
+        torch.bfloat16).view(torch.int16)
+    x_swa = torch.randn((L, B, 512), generator=g, device=dev).to(torch.bfloat16).view(torch.int16)
+    swa = torch.zeros((L, B, 128, 512), dtype=torch.uint8, device=dev)
+    swa_pos = torch.zeros(B, dtype=torch.int32, device=dev)
+    swa_len = torch.zeros(B, dtype=torch.int32, device=dev)
+    ws = csa2.workspace(csa2.WS_HEADER, device=dev)
+
+    def call():
+        csa2.csa2_cache_append(kv, x, w_idx, ws, x_swa, swa, swa_pos, swa_len)
+
+    for _ in range(W):
+        call()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    csa2.csa2_sync_status(ws)
+    assert int(n_rows.min()) == W + K and int(swa_pos.min()) == W + K
+    us = 1e3 * e0.elapsed_time(e1) / K
+    per_seq = 1024 + 256 + 32 + 128 + L * (1024 + 512)
+    return {"us_per_call": us, "launches_per_call": 2, "batch": B, "layers": L,
+            "algorithmic_bytes_per_call": B * per_seq + 512 * 64 * 2,
+            "timing": f"{K} back-to-back calls after {W} warm-up calls, CUDA events"}
+
+
 def run_gpu(args, wl, rank, world):
     import torch
 
@@ -333,6 +378,8 @@ def run_gpu(args, wl, rank, world):
     barrier()
     t_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / K, dist, dev)
 
+    append = time_cache_append(csa2, wl, dev, stream, K, args.warmup)
+
     units = wl.B * wl.L
     value = job_throughput(units, world, t_step)
     ab = algorithmic_bytes(wl)
@@ -361,6 +408,7 @@ def run_gpu(args, wl, rank, world):
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(units, world, t_e2e), "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "next_rows": {"cache_append": append},
             "gpu_launches": int(launches * K),
             "gpu_launches_per_step": int(launches),
             "clocks": sampler.summary(),
