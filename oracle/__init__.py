@@ -90,6 +90,12 @@ def lib():
                                         C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
                                         C.c_int32, C.c_double, C.c_void_p, C.c_void_p,
                                         C.c_void_p, C.c_void_p, C.c_void_p]
+        L.csa2o_layer_group_multi.argtypes = [C.POINTER(_KV), C.POINTER(_Dims), C.c_int32,
+                                              C.c_int32, C.c_void_p, C.c_int32, C.c_void_p,
+                                              C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                              C.c_void_p, C.c_int32, C.c_int32, C.c_double,
+                                              C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                              C.c_void_p]
         L.csa2o_project_idxk.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
                                          C.c_void_p]
         L.csa2o_cache_append.argtypes = [C.POINTER(_KV), C.POINTER(_Dims), C.c_int32,
@@ -292,3 +298,37 @@ def cache_append(kv: KV, dm, n_rows: np.ndarray, x: np.ndarray, w_idx: np.ndarra
                                     _p(kv.idxk), _p(n_rows), _p(x), _p(w_idx), L,
                                     _p(x_swa) if L else None, _p(swa) if L else None,
                                     _p(swa_pos) if L else None, _p(swa_len) if L else None)
+
+
+# ------------------------------------------------ multi-query decode (next row)
+def layer_group_multi(kv: KV, dm, n_rows, n_query: int, modes, q_idx, w, q, swa, swa_len, *,
+                      top_k=512, pool_blocks=2048, sm_scale=None):
+    """Q = n_query draft positions per sequence in one step.  Inputs carry a
+    query axis after the batch axis (q_idx [L][B][Q][8][64], w [L][B][Q][8],
+    q [L][B][Q][16][512]); the window is swa [L][B][128 + Q - 1][512] with
+    swa_len [B].  Returns dict(idx [L][B][Q][k], idx_count [L][B][Q],
+    pool [B][Q][pool_blocks], pool_count [B][Q], out [L][B][Q][16][512])."""
+    n_rows = _c(n_rows, np.int64)
+    modes = _c(modes, np.int32)
+    q_idx = _c(q_idx, np.uint16)
+    w = _c(w, np.float32)
+    q = _c(q, np.uint16)
+    swa = _c(swa, np.uint8)
+    swa_len = _c(swa_len, np.int32)
+    B, L, Q = len(n_rows), len(modes), int(n_query)
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(dm.d)
+    idx = np.full((L, B, Q, top_k), -1, np.int32)
+    idx_count = np.zeros((L, B, Q), np.int32)
+    pb = max(pool_blocks, 1)
+    pool_ = np.full((B, Q, pb), -1, np.int32)
+    pool_count = np.zeros((B, Q), np.int32)
+    out = np.zeros((L, B, Q, dm.h, dm.d), np.float64)
+    rc = lib().csa2o_layer_group_multi(C.byref(kv.s), C.byref(dm), B, Q, _p(n_rows), L,
+                                       _p(modes), _p(q_idx), _p(w), _p(q), _p(swa), _p(swa_len),
+                                       top_k, pool_blocks, sm_scale, _p(idx), _p(idx_count),
+                                       _p(pool_), _p(pool_count), _p(out))
+    if rc:
+        raise ValueError("oracle multi-query layer group: bad arguments or row outside the pool")
+    return dict(idx=idx, idx_count=idx_count, pool=pool_[..., :pool_blocks],
+                pool_count=pool_count, out=out)

@@ -423,3 +423,78 @@ int csa2o_cache_append(const csa2o_kv *kv, const csa2o_dims *dm, int32_t B,
   }
   return rc;
 }
+
+/* ----------------------------------------------------- multi-query decode */
+
+int csa2o_layer_group_multi(const csa2o_kv *kv, const csa2o_dims *dm, int32_t B, int32_t Q,
+                            const int64_t *n_rows, int32_t L, const int32_t *modes,
+                            const uint16_t *q_idx, const float *w, const uint16_t *q,
+                            const uint8_t *swa, const int32_t *swa_len, int32_t top_k,
+                            int32_t pool_blocks, double sm_scale, int32_t *idx,
+                            int32_t *idx_count, int32_t *pool, int32_t *pool_count,
+                            double *out) {
+  if (B < 0 || Q < 1 || L < 0 || top_k < 1) return CSA2O_EARG;
+  const int HI = dm->hi, DI = dm->di, H = dm->h, D = dm->d, W = dm->w;
+  const int64_t WR = (int64_t)W + Q - 1; /* window rows per (layer, sequence) */
+  const int pb = pool_blocks > 0 ? pool_blocks : 1;
+  uint16_t *qi_t = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(L ? L : 1) * HI * DI);
+  float *w_t = (float *)malloc(sizeof(float) * (size_t)(L ? L : 1) * HI);
+  uint16_t *q_t = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(L ? L : 1) * H * D);
+  uint8_t *swa_t = (uint8_t *)calloc((size_t)(L ? L : 1) * W * D, 1);
+  int32_t *idx_t = (int32_t *)malloc(sizeof(int32_t) * (size_t)(L ? L : 1) * top_k);
+  int32_t *cnt_t = (int32_t *)malloc(sizeof(int32_t) * (size_t)(L ? L : 1));
+  int32_t *pool_t = (int32_t *)malloc(sizeof(int32_t) * (size_t)pb);
+  double *out_t = (double *)malloc(sizeof(double) * (size_t)(L ? L : 1) * H * D);
+  int rc = CSA2O_OK;
+  for (int32_t b = 0; b < B && rc == CSA2O_OK; b++) {
+    /* the view of sequence b alone, as batch entry 0 */
+    csa2o_kv one = *kv;
+    if (kv->page_table) {
+      one.page_table = kv->page_table + (int64_t)b * kv->max_pages;
+    } else {
+      const int64_t off = (int64_t)b * kv->seq_stride;
+      one.codes = kv->codes + off * (D / 2);
+      one.scales = kv->scales + off * (D / 16);
+      one.idxk = kv->idxk + off * DI;
+      one.pool_rows = kv->pool_rows - off;
+    }
+    for (int32_t t = 0; t < Q && rc == CSA2O_OK; t++) {
+      const int64_t v = (int64_t)b * Q + t; /* (b, t) on the flattened axis */
+      int64_t C = n_rows[b] - (Q - 1 - t);
+      if (C < 0) C = 0;
+      int64_t e = (int64_t)swa_len[b] - (Q - 1 - t);
+      if (e < 0) e = 0;
+      const int64_t s0 = e > W ? e - W : 0;
+      const int32_t len = (int32_t)(e - s0);
+      for (int32_t l = 0; l < L; l++) {
+        memcpy(qi_t + (size_t)l * HI * DI, q_idx + ((size_t)l * B * Q + v) * HI * DI,
+               sizeof(uint16_t) * HI * DI);
+        memcpy(w_t + (size_t)l * HI, w + ((size_t)l * B * Q + v) * HI, sizeof(float) * HI);
+        memcpy(q_t + (size_t)l * H * D, q + ((size_t)l * B * Q + v) * H * D,
+               sizeof(uint16_t) * H * D);
+        memcpy(swa_t + (size_t)l * W * D, swa + (((size_t)l * B + b) * WR + s0) * D,
+               (size_t)len * D);
+      }
+      rc = csa2o_layer_group(&one, dm, 1, &C, L, modes, qi_t, w_t, q_t, swa_t, &len, top_k,
+                             pool_blocks, sm_scale, idx_t, cnt_t, pool_t, pool_count + v, out_t);
+      for (int32_t l = 0; l < L; l++) {
+        memcpy(idx + ((size_t)l * B * Q + v) * top_k, idx_t + (size_t)l * top_k,
+               sizeof(int32_t) * top_k);
+        idx_count[(size_t)l * B * Q + v] = cnt_t[l];
+        memcpy(out + ((size_t)l * B * Q + v) * H * D, out_t + (size_t)l * H * D,
+               sizeof(double) * H * D);
+      }
+      if (pool_blocks > 0)
+        memcpy(pool + (size_t)v * pool_blocks, pool_t, sizeof(int32_t) * pool_blocks);
+    }
+  }
+  free(qi_t);
+  free(w_t);
+  free(q_t);
+  free(swa_t);
+  free(idx_t);
+  free(cnt_t);
+  free(pool_t);
+  free(out_t);
+  return rc;
+}

@@ -160,6 +160,28 @@ int csa2o_attention(const csa2o_kv *kv, const csa2o_dims *dm, int32_t b,
                     int32_t n_idx, const uint8_t *swa /*[w][d]*/,
                     int32_t swa_len, double sm_scale, double *out /*[h][d]*/);
 
+/* ------------------------------ multi-query decode (next row of work) */
+
+/* Verification of Q draft positions in one step (the drafts' entries are
+ * already in the caches): query t < Q of sequence b is one decode step that
+ * sees the first C_t = n_rows[b] - (Q - 1 - t) global entries (fewer than 0
+ * means none) and the window rows [max(0, e_t - w), e_t) of its layer, with
+ * e_t = swa_len[b] - (Q - 1 - t).  Per-query inputs and outputs carry a query
+ * axis after the batch axis: q_idx [L][B][Q][hi][di], w [L][B][Q][hi],
+ * q [L][B][Q][h][d], idx [L][B][Q][top_k], idx_count [L][B][Q],
+ * pool [B][Q][pool_blocks], pool_count [B][Q], out [L][B][Q][h][d]; the
+ * window is swa [L][B][w + Q - 1][d] with swa_len[B] <= w + Q - 1 valid rows.
+ * Each (b, t) is computed by csa2o_layer_group on its own truncated view.
+ * [CNB / REL: DSpark drafts several positions and the main model verifies
+ * them in one pass]; causal visibility among drafts is this build's reading. */
+int csa2o_layer_group_multi(const csa2o_kv *kv, const csa2o_dims *dm, int32_t B, int32_t Q,
+                            const int64_t *n_rows, int32_t L, const int32_t *modes,
+                            const uint16_t *q_idx, const float *w, const uint16_t *q,
+                            const uint8_t *swa, const int32_t *swa_len, int32_t top_k,
+                            int32_t pool_blocks, double sm_scale, int32_t *idx,
+                            int32_t *idx_count, int32_t *pool, int32_t *pool_count,
+                            double *out);
+
 /* --------------------------------------- cache append (next row of work) */
 
 /* Indexer-K projection of one main-KV entry:
