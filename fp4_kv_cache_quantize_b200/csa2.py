@@ -50,7 +50,7 @@ class GroupDesc(C.Structure):
                 ("swa", C.c_void_p), ("swa_len", C.c_void_p), ("top_k", C.c_int32),
                 ("pool_blocks", C.c_int32), ("sm_scale", C.c_float), ("idx", C.c_void_p),
                 ("idx_count", C.c_void_p), ("pool", C.c_void_p), ("pool_count", C.c_void_p),
-                ("out", C.c_void_p)]
+                ("out", C.c_void_p), ("n_query", C.c_int32)]
 
 
 class TraceStruct(C.Structure):
@@ -218,12 +218,14 @@ def csa2_cache_append(kv: KVCache, x, w_idx, ws, x_swa=None, swa=None, swa_pos=N
 
 
 class LayerGroup:
-    """A csa2_group_desc over device tensors (kept alive by this object)."""
+    """A csa2_group_desc over device tensors (kept alive by this object).
+    With n_query = Q > 1 every per-query array has batch x Q rows (query axis
+    after the batch axis) and swa holds 128 + Q - 1 rows per sequence."""
 
     def __init__(self, kv: KVCache, modes, q_idx, w, q, swa, swa_len, *, top_k=512,
                  pool_blocks=2048, sm_scale=None, idx=None, idx_count=None, pool=None,
-                 pool_count=None, out=None):
-        L, B = len(modes), kv.batch
+                 pool_count=None, out=None, n_query=1):
+        L, B = len(modes), kv.batch * max(int(n_query), 1)
         dev = q.device
         self.kv = kv
         self.modes_host = (C.c_int32 * L)(*[int(m) for m in modes])
@@ -246,7 +248,7 @@ class LayerGroup:
                               _ptr(w), _ptr(q), _ptr(swa), _ptr(self.swa_len), top_k,
                               pool_blocks, float(sm_scale), _ptr(self.idx),
                               _ptr(self.idx_count), _ptr(self.pool), _ptr(self.pool_count),
-                              _ptr(self.out))
+                              _ptr(self.out), int(n_query))
 
     def workspace_size(self) -> int:
         return _group_ws(C.byref(self.desc))

@@ -99,22 +99,30 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
   const int g = lane >> 2, tig = lane & 3;
   const uint32_t q_base = smem_u32(s.q), kv_base = smem_u32(s.kv), p_base = smem_u32(s.p);
 
-  int C = p.n_rows[b];
+  // b runs over sequences x queries: query tq of sequence bp sees the
+  // sequence's entries minus the drafts after it, and the window rows that
+  // end at its own entry.
+  const int bp = b / p.nq, tq = b - bp * p.nq, later = p.nq - 1 - tq;
+  int C = p.n_rows[bp];
   if (C < 0 || C > p.max_rows) {
     set_status(p.status, ST_DEVICE_CHECK);
     C = C < 0 ? 0 : p.max_rows;
   }
+  C = C - later < 0 ? 0 : C - later;
   int n_idx = L.idx_count[b];
   if (n_idx < 0 || n_idx > p.idx_stride) {
     set_status(p.status, ST_DEVICE_CHECK);
     n_idx = n_idx < 0 ? 0 : p.idx_stride;
   }
   if (n_idx > CSA2_MAX_TOPK) n_idx = CSA2_MAX_TOPK;
-  int n_swa = p.swa_len[b];
-  if (n_swa < 0 || n_swa > CSA2_W) {
+  int n_win = p.swa_len[bp];
+  if (n_win < 0 || n_win > p.swa_rows) {
     set_status(p.status, ST_DEVICE_CHECK);
-    n_swa = n_swa < 0 ? 0 : CSA2_W;
+    n_win = n_win < 0 ? 0 : p.swa_rows;
   }
+  const int win_end = n_win - later < 0 ? 0 : n_win - later;
+  const int win_lo = win_end > CSA2_W ? win_end - CSA2_W : 0;
+  const int n_swa = win_end - win_lo;
   const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
 
   if (split == 0 && L.idx_copy) {  // Reuse layer: publish the indices it used
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
       if (k0 + t < nk) {
         if (sparse) {
           const int pos = __ldg(idx + k0 + t);
-          if (pos >= 0 && pos < C) row = kv_row(p, b, pos);
+          if (pos >= 0 && pos < C) row = kv_row(p, bp, pos);
           if (row < 0) set_status(p.status, ST_DEVICE_CHECK);
         } else {
           row = k0 + t;
@@ -189,7 +197,7 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
         int64_t row = -1;
         if (k0 + r < nk) {
           const int pos = __ldg(idx + k0 + r);
-          if (pos >= 0 && pos < C) row = kv_row(p, b, pos);
+          if (pos >= 0 && pos < C) row = kv_row(p, bp, pos);
         }
         if (row >= 0) {
           cv[u] = __ldg(reinterpret_cast<const uint4*>(p.codes + row * (CSA2_D / 2)) + cc);
@@ -224,7 +232,7 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
       }
     } else {
       // 64 window rows x 32 chunks of 16 E4M3 bytes.
-      const uint8_t* swa = L.swa + (int64_t)b * CSA2_W * CSA2_D;
+      const uint8_t* swa = L.swa + ((int64_t)bp * p.swa_rows + win_lo) * CSA2_D;
       uint4 cv[16];
 #pragma unroll
       for (int u = 0; u < 16; u++) {

@@ -112,8 +112,10 @@ struct IndexWs {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-static IndexWs index_ws_layout(const csa2_kv_view* kv, int top_k, uint8_t* base) {
+// nq queries per sequence: block maxima and candidates per (sequence, query).
+static IndexWs index_ws_layout(const csa2_kv_view* kv, int top_k, uint8_t* base, int nq = 1) {
   IndexWs w{};
+  const size_t vb = (size_t)kv->batch * nq;
   const int nblk = (kv->max_rows + CSA2_BLK - 1) / CSA2_BLK;
   w.bm_stride = ((nblk + 15) / 16) * 16;
   if (w.bm_stride == 0) w.bm_stride = 16;
@@ -121,16 +123,17 @@ static IndexWs index_ws_layout(const csa2_kv_view* kv, int top_k, uint8_t* base)
   size_t off = CSA2_WS_HEADER;
   w.status = reinterpret_cast<uint32_t*>(base);
   w.bm = reinterpret_cast<float*>(base + off);
-  off = align256(off + (size_t)kv->batch * w.bm_stride * sizeof(float));
+  off = align256(off + vb * w.bm_stride * sizeof(float));
   w.sel = reinterpret_cast<int32_t*>(base + off);
-  off = align256(off + (size_t)kv->batch * w.sel_stride * sizeof(int32_t));
+  off = align256(off + vb * w.sel_stride * sizeof(int32_t));
   w.sel_count = reinterpret_cast<int32_t*>(base + off);
-  off = align256(off + (size_t)kv->batch * sizeof(int32_t));
+  off = align256(off + vb * sizeof(int32_t));
   w.bytes = off;
   return w;
 }
 
-static ScanParams scan_params(const csa2_kv_view* kv, const float* w, const IndexWs& ws) {
+static ScanParams scan_params(const csa2_kv_view* kv, const float* w, const IndexWs& ws,
+                              int nq) {
   ScanParams p{};
   p.n_rows = kv->n_rows;
   p.page_table = kv->page_table;
@@ -143,14 +146,16 @@ static ScanParams scan_params(const csa2_kv_view* kv, const float* w, const Inde
   p.bm_stride = ws.bm_stride;
   p.batch = kv->batch;
   p.tiles_per_seq = (kv->max_rows + SC_TILE - 1) / SC_TILE;
+  p.nq = nq;
   p.status = ws.status;
   return p;
 }
 
 static RescoreParams rescore_params(const csa2_kv_view* kv, const int32_t* cand,
                                     const int32_t* cand_count, int cand_stride, int top_k,
-                                    uint32_t* status) {
+                                    uint32_t* status, int nq = 1) {
   RescoreParams p{};
+  p.nq = nq;
   p.idx_k = kv->idx_k;
   p.page_table = kv->page_table;
   p.max_pages = kv->max_pages;
@@ -169,17 +174,17 @@ static RescoreParams rescore_params(const csa2_kv_view* kv, const int32_t* cand,
 // scan + block select: candidates (top P blocks by block max) into sel
 static csa2_status run_scan_select(const csa2_kv_view* kv, const uint16_t* q_idx, const float* w,
                                    int P, int32_t* sel, int32_t* sel_count, int sel_stride,
-                                   const IndexWs& ws, cudaStream_t st) {
+                                   const IndexWs& ws, cudaStream_t st, int nq = 1) {
   CUtensorMap map_k, map_q;
   csa2_status r = map_rows64(&map_k, kv->idx_k, (uint64_t)kv->pool_rows, 64);
   if (r) return r;
-  r = map_rows64(&map_q, q_idx, (uint64_t)kv->batch * CSA2_HI, 16);
+  r = map_rows64(&map_q, q_idx, (uint64_t)kv->batch * nq * CSA2_HI, scan_query_rows(nq));
   if (r) return r;
   trace_mark("scan", st);
-  CSA2_CUDA(launch_scan(map_k, map_q, scan_params(kv, w, ws), num_sms(), st));
+  CSA2_CUDA(launch_scan(map_k, map_q, scan_params(kv, w, ws, nq), num_sms(), st));
   trace_mark("block_select", st);
-  CSA2_CUDA(launch_block_select(ws.bm, ws.bm_stride, kv->n_rows, kv->max_rows, kv->batch, P, sel,
-                                sel_stride, sel_count, ws.status, st));
+  CSA2_CUDA(launch_block_select(ws.bm, ws.bm_stride, kv->n_rows, kv->max_rows, kv->batch * nq, nq,
+                                P, sel, sel_stride, sel_count, ws.status, st));
   return CSA2_OK;
 }
 
@@ -197,14 +202,17 @@ struct GroupWs {
   size_t bytes;
 };
 
+static int group_nq(const csa2_group_desc* d) { return d->n_query < 1 ? 1 : d->n_query; }
+
 static GroupWs group_ws_layout(const csa2_group_desc* d, uint8_t* base) {
   GroupWs g{};
-  g.ix = index_ws_layout(&d->kv, d->top_k, base);
-  g.nsplit = attn_nsplit(d->kv.batch * d->n_layers, num_sms());
-  const size_t slots = (size_t)d->kv.batch * d->n_layers * g.nsplit;
+  const int nq = group_nq(d), vb = d->kv.batch * nq;
+  g.ix = index_ws_layout(&d->kv, d->top_k, base, nq);
+  g.nsplit = attn_nsplit(vb * d->n_layers, num_sms());
+  const size_t slots = (size_t)vb * d->n_layers * g.nsplit;
   g.part_o = reinterpret_cast<float*>(base + g.ix.bytes);
   g.part_ml = reinterpret_cast<float*>(base + g.ix.bytes + slots * CSA2_H * CSA2_D * sizeof(float));
-  g.bytes = g.ix.bytes + align256(attn_partial_bytes(d->kv.batch, d->n_layers, g.nsplit));
+  g.bytes = g.ix.bytes + align256(attn_partial_bytes(vb, d->n_layers, g.nsplit));
   return g;
 }
 
@@ -299,8 +307,10 @@ size_t csa2_attn_workspace_size(int32_t batch, int32_t n_layers) {
 }
 
 static csa2_status fill_attn_common(AttnParams& ap, const csa2_kv_view* kv, const int32_t* swa_len,
-                                    float sm_scale, int idx_stride) {
-  ap.batch = kv->batch;
+                                    float sm_scale, int idx_stride, int nq = 1) {
+  ap.batch = kv->batch * nq;
+  ap.nq = nq;
+  ap.swa_rows = CSA2_W + nq - 1;
   ap.idx_stride = idx_stride;
   ap.codes = kv->codes;
   ap.scales = kv->scales;
@@ -361,7 +371,10 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
   csa2_status r = check_kv(kv);
   if (r) return r;
   if ((r = check_topk(d->top_k, d->pool_blocks))) return r;
-  const int L = d->n_layers, B = kv->batch;
+  const int L = d->n_layers, B = kv->batch, nq = group_nq(d), VB = B * nq;
+  CSA2_REQUIRE(d->n_query >= 0 && d->n_query <= CSA2_MAX_QUERY, CSA2_ERR_SHAPE,
+               "n_query = %d outside [0, %d]", d->n_query, (int)CSA2_MAX_QUERY);
+  CSA2_REQUIRE(VB <= 65535, CSA2_ERR_SHAPE, "batch x n_query = %d > 65535", VB);
   CSA2_REQUIRE(L >= 1 && L <= AT_MAX_LAYERS, CSA2_ERR_SHAPE, "n_layers = %d outside [1, %d]", L,
                AT_MAX_LAYERS);
   CSA2_REQUIRE(d->modes != nullptr, CSA2_ERR_INVALID_ARG, "modes is NULL");
@@ -389,9 +402,9 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
                g.bytes);
   cudaStream_t st = (cudaStream_t)stream;
   const int K = d->top_k;
-  const size_t qi_stride = (size_t)B * CSA2_HI * CSA2_DI, w_stride = (size_t)B * CSA2_HI;
-  auto layer_idx = [&](int l) { return d->idx + (size_t)l * B * K; };
-  auto layer_cnt = [&](int l) { return d->idx_count + (size_t)l * B; };
+  const size_t qi_stride = (size_t)VB * CSA2_HI * CSA2_DI, w_stride = (size_t)VB * CSA2_HI;
+  auto layer_idx = [&](int l) { return d->idx + (size_t)l * VB * K; };
+  auto layer_cnt = [&](int l) { return d->idx_count + (size_t)l * VB; };
 
   // Indexer: per FULL layer, one scan + block select and one rescore launch
   // for the FULL layer and the REINDEX layers that share its pool.
@@ -405,8 +418,8 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
     int32_t* sel = hsi ? d->pool : g.ix.sel;
     int32_t* sel_count = hsi ? d->pool_count : g.ix.sel_count;
     const int sel_stride = hsi ? d->pool_blocks : g.ix.sel_stride;
-    if ((r = run_scan_select(kv, qi, wl, P, sel, sel_count, sel_stride, g.ix, st))) return r;
-    RescoreParams rp = rescore_params(kv, sel, sel_count, sel_stride, K, g.ix.status);
+    if ((r = run_scan_select(kv, qi, wl, P, sel, sel_count, sel_stride, g.ix, st, nq))) return r;
+    RescoreParams rp = rescore_params(kv, sel, sel_count, sel_stride, K, g.ix.status, nq);
     int nj = 0;
     rp.job[nj++] = RescoreJob{qi, wl, layer_idx(l), layer_cnt(l), K};
     if (hsi && d->modes[l] == CSA2_FULL) {
@@ -414,7 +427,7 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
         if (d->modes[x] != CSA2_REINDEX) continue;
         if (nj == RS_MAX_JOBS) {
           trace_mark("rescore", st);
-  CSA2_CUDA(launch_rescore(rp, nj, B, cand_blocks_max(kv, P), st));
+          CSA2_CUDA(launch_rescore(rp, nj, VB, cand_blocks_max(kv, P), st));
           nj = 0;
         }
         rp.job[nj++] =
@@ -422,12 +435,12 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
       }
     }
     trace_mark("rescore", st);
-  CSA2_CUDA(launch_rescore(rp, nj, B, cand_blocks_max(kv, P), st));
+    CSA2_CUDA(launch_rescore(rp, nj, VB, cand_blocks_max(kv, P), st));
   }
 
   // Attention for every layer in one launch.
   AttnParams ap{};
-  fill_attn_common(ap, kv, d->swa_len, d->sm_scale, K);
+  fill_attn_common(ap, kv, d->swa_len, d->sm_scale, K, nq);
   ap.n_layers = L;
   ap.nsplit = g.nsplit;
   ap.part_o = g.part_o;
@@ -437,13 +450,13 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
   for (int l = 0; l < L; l++) {
     if (d->modes[l] != CSA2_REUSE) src = l;
     const bool reuse = d->modes[l] == CSA2_REUSE;
-    ap.layer[l] = AttnLayer{d->q + (size_t)l * B * CSA2_H * CSA2_D,
-                            d->swa + (size_t)l * B * CSA2_W * CSA2_D,
+    ap.layer[l] = AttnLayer{d->q + (size_t)l * VB * CSA2_H * CSA2_D,
+                            d->swa + (size_t)l * B * ap.swa_rows * CSA2_D,
                             layer_idx(src),
                             layer_cnt(src),
                             reuse ? layer_idx(l) : nullptr,
                             reuse ? layer_cnt(l) : nullptr,
-                            d->out + (size_t)l * B * CSA2_H * CSA2_D};
+                            d->out + (size_t)l * VB * CSA2_H * CSA2_D};
   }
   CSA2_CUDA(launch_attn(ap, st));
   trace_mark("end", st);

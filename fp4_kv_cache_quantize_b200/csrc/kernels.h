@@ -24,6 +24,7 @@ struct ScanParams {
   int32_t bm_stride;
   int32_t batch;
   int32_t tiles_per_seq;
+  int32_t nq;        // queries per sequence; w and bm are [batch * nq][...]
   uint32_t* status;
 };
 constexpr int SC_TILE = 128;
@@ -49,6 +50,7 @@ struct RescoreParams {
   const int32_t* cand_count;
   int32_t cand_stride;
   int32_t top_k;
+  int32_t nq;        // queries per sequence: blockIdx.y runs over batch * nq
   uint32_t* status;
 };
 
@@ -56,9 +58,12 @@ cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, cons
                         int num_sms, cudaStream_t st);
 cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
                            cudaStream_t st);
+// batch counts sequences x queries (nq per sequence).
 cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n_rows,
-                                int max_rows, int batch, int k_req, int32_t* sel, int sel_stride,
-                                int32_t* sel_count, uint32_t* status, cudaStream_t st);
+                                int max_rows, int batch, int nq, int k_req, int32_t* sel,
+                                int sel_stride, int32_t* sel_count, uint32_t* status,
+                                cudaStream_t st);
+int scan_query_rows(int nq);
 
 // attn.cu --------------------------------------------------------------
 constexpr int AT_MAX_LAYERS = 32;
@@ -84,6 +89,8 @@ struct AttnParams {
   const int32_t* n_rows;
   const int32_t* swa_len;
   float scale_log2;
+  int32_t nq;        // queries per sequence: blockIdx.y runs over batch * nq
+  int32_t swa_rows;  // window rows per (layer, sequence): 128 + nq - 1
   float* part_o;   // [n_layers][batch][nsplit][16][512] split partials (nsplit > 1)
   float* part_ml;  // [n_layers][batch][nsplit][16][2] their max and sum
   uint32_t* status;

@@ -28,25 +28,31 @@ namespace csa2 {
 
 // ------------------------------------------------------------- the scan
 constexpr int SC_BOX = 64;                 // rows per TMA box
-constexpr int SC_N = 16;                   // indexer heads padded to MMA N
 constexpr int SC_STAGES = 3;
-constexpr int SC_CTAS_PER_SM = 4;          // four independent pipelines per SM
-constexpr int SC_ACC = 4;                  // TMEM accumulator buffers (16 columns each)
+constexpr int SC_CTAS_PER_SM = 4;          // up to four independent pipelines per SM
 constexpr int SC_A_BYTES = SC_TILE * 128;  // 16 KB of indexer K per stage
-constexpr int SC_B_BYTES = SC_N * 128;     // 2 KB of indexer query per stage
 constexpr int SC_THREADS = 192;            // producer, MMA, 4 epilogue warps
-constexpr uint32_t SC_IDESC = idesc_bf16_f32(SC_TILE, SC_N);
 
-struct ScanSmem {
-  uint8_t a[SC_STAGES][SC_A_BYTES];
-  uint8_t b[SC_STAGES][SC_B_BYTES];
-  uint64_t full[SC_STAGES], empty[SC_STAGES];
-  uint64_t tfull[SC_ACC], tempty[SC_ACC], done;
-  uint32_t tmem_base;
-  int abort;
+// One instantiation per MMA width N: the 8 indexer heads of every query of a
+// sequence (nq queries, 8 nq <= N), padded to 16, 32 or 64; ACC accumulators
+// of N fp32 columns in TMEM.
+template <int N, int ACC>
+struct ScanCfg {
+  static constexpr int B_BYTES = N * 128;  // indexer queries per stage
+  static constexpr uint32_t IDESC = idesc_bf16_f32(SC_TILE, N);
+  static constexpr uint32_t TMEM_COLS = N * ACC;
+  static_assert(TMEM_COLS >= 32 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation size");
+  static_assert(TMEM_COLS * SC_CTAS_PER_SM <= 512, "TMEM columns of one SM");
+  struct Smem {
+    uint8_t a[SC_STAGES][SC_A_BYTES];
+    uint8_t b[SC_STAGES][B_BYTES];
+    uint64_t full[SC_STAGES], empty[SC_STAGES];
+    uint64_t tfull[ACC], tempty[ACC], done;
+    uint32_t tmem_base;
+    int abort;
+  };
+  static constexpr size_t SMEM = sizeof(Smem) + 1024;
 };
-constexpr size_t SC_SMEM = sizeof(ScanSmem) + 1024;
-
 
 __device__ __forceinline__ int visible_rows(const int32_t* n_rows, int b, int max_rows,
                                             uint32_t* status) {
@@ -56,6 +62,15 @@ __device__ __forceinline__ int visible_rows(const int32_t* n_rows, int b, int ma
     c = c < 0 ? 0 : max_rows;
   }
   return c;
+}
+
+// Entries visible to query v % nq of sequence v / nq: the sequence's count
+// minus the drafts after that query (never negative).
+__device__ __forceinline__ int visible_query(const int32_t* n_rows, int v, int nq, int max_rows,
+                                             uint32_t* status) {
+  const int b = v / nq, t = v - b * nq;
+  const int c = visible_rows(n_rows, b, max_rows, status) - (nq - 1 - t);
+  return c < 0 ? 0 : c;
 }
 
 // First pool row of the 64-row box holding position pos0 (a multiple of 64),
@@ -77,9 +92,12 @@ __device__ __forceinline__ int32_t box_row(const ScanParams& p, int b, int pos0)
   return (int32_t)row;
 }
 
-__global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
+template <int N, int ACC>
+__global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
     score_scan_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_q, const ScanParams p) {
+  using Cfg = ScanCfg<N, ACC>;
+  using ScanSmem = typename Cfg::Smem;
   extern __shared__ uint8_t smem_raw[];
   ScanSmem& s = *reinterpret_cast<ScanSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -92,7 +110,7 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int i = 0; i < SC_ACC; i++) {
+    for (int i = 0; i < ACC; i++) {
       mbar_init(&s.tfull[i], 1);
       mbar_init(&s.tempty[i], 4 * 32);
     }
@@ -103,7 +121,7 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
     tma_prefetch_desc(&map_q);
   }
   if (warp == 1) {
-    tmem_alloc(&s.tmem_base, SC_ACC * SC_N);  // SC_ACC 16-column fp32 accumulators
+    tmem_alloc(&s.tmem_base, Cfg::TMEM_COLS);  // ACC accumulators of N fp32 columns
     tmem_relinquish();
   }
   tc_fence_before();
@@ -131,10 +149,10 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
         const int pos0 = t * SC_TILE;
         const int32_t y0 = box_row(p, b, pos0);
         const int32_t y1 = pos0 + SC_BOX < C ? box_row(p, b, pos0 + SC_BOX) : y0;
-        mbar_arrive_expect_tx(&s.full[stage], SC_A_BYTES + SC_B_BYTES);
+        mbar_arrive_expect_tx(&s.full[stage], SC_A_BYTES + Cfg::B_BYTES);
         tma_load_2d(s.a[stage], &map_k, &s.full[stage], 0, y0);
         tma_load_2d(s.a[stage] + SC_BOX * 128, &map_k, &s.full[stage], 0, y1);
-        tma_load_2d(s.b[stage], &map_q, &s.full[stage], 0, b * CSA2_HI);
+        tma_load_2d(s.b[stage], &map_q, &s.full[stage], 0, b * CSA2_HI * p.nq);
         issued |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == SC_STAGES) {
@@ -167,10 +185,10 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
         }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(s.a[stage]), b_addr = smem_u32(s.b[stage]);
-        const uint32_t d = tmem + (uint32_t)(acc * SC_N);
+        const uint32_t d = tmem + (uint32_t)(acc * N);
 #pragma unroll
         for (int k = 0; k < 4; k++)  // K = 64 as four K = 16 steps inside the swizzle atom
-          umma_bf16(d, sdesc_k128(a_addr + 32 * k), sdesc_k128(b_addr + 32 * k), SC_IDESC,
+          umma_bf16(d, sdesc_k128(a_addr + 32 * k), sdesc_k128(b_addr + 32 * k), Cfg::IDESC,
                     k > 0);
         umma_commit(&s.empty[stage]);
         umma_commit(&s.tfull[acc]);
@@ -178,7 +196,7 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
           stage = 0;
           phase ^= 1u;
         }
-        if (++acc == SC_ACC) {
+        if (++acc == ACC) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -187,18 +205,20 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
       if (!mbar_wait(&s.done, 0, nullptr)) set_status(p.status, ST_TIMEOUT);
     }
   } else {  // ------------------------------------------ epilogue, 4 warps
+    // Thread = one TMEM lane = one position of the tile.  Query tq's score
+    // is the weighted ReLU sum over accumulator columns [8 tq, 8 tq + 8).
+    constexpr int QPB = N / 8 < 4 ? N / 8 : 4;  // queries per batch of TMEM loads
     const int quarter = warp & 3;  // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
+    const int nq = p.nq;
     int acc = 0;
     uint32_t acc_phase = 0;
-    int cur_b = -1, C = 0;
-    float w[CSA2_HI];
+    int cur_b = -1, C = 0, w_b = -1, w_t0 = -1;
+    float wr[QPB][CSA2_HI];
     for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
       const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
       if (b != cur_b) {
-        C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
-#pragma unroll
-        for (int h = 0; h < CSA2_HI; h++) w[h] = __ldg(p.w + b * CSA2_HI + h);
+        C = visible_rows(p.n_rows, b, p.max_rows, nullptr);  // the last query's view
         cur_b = b;
       }
       if (t * SC_TILE >= C) continue;
@@ -209,21 +229,46 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
         break;
       }
       tc_fence_after();
-      uint32_t r[8];
-      tmem_ld_x8(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * SC_N), r);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s.tempty[acc]);
-      float sc = 0.0f;
-#pragma unroll
-      for (int h = 0; h < CSA2_HI; h++) sc = fmaf(w[h], fmaxf(__uint_as_float(r[h]), 0.0f), sc);
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
       const int pos = t * SC_TILE + row;
-      if (pos >= C) sc = -INFINITY;
-      sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
-      sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
-      sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
-      if ((lane & 7) == 0 && pos < C) p.bm[(int64_t)b * p.bm_stride + pos / CSA2_BLK] = sc;
-      if (++acc == SC_ACC) {
+      for (int t0 = 0; t0 < nq; t0 += QPB) {
+        uint32_t r[QPB][8];
+#pragma unroll
+        for (int qq = 0; qq < QPB; qq++)
+          if (t0 + qq < nq) tmem_ld_x8(tbase + (uint32_t)(8 * (t0 + qq)), r[qq]);
+        tmem_ld_wait();
+        if (t0 + QPB >= nq) {  // every load of this accumulator has completed
+          tc_fence_before();
+          mbar_arrive(&s.tempty[acc]);
+        }
+        if (b != w_b || t0 != w_t0) {
+#pragma unroll
+          for (int qq = 0; qq < QPB; qq++)
+#pragma unroll
+            for (int h = 0; h < CSA2_HI; h++)
+              wr[qq][h] = t0 + qq < nq ? __ldg(p.w + ((int64_t)b * nq + t0 + qq) * CSA2_HI + h)
+                                       : 0.0f;
+          w_b = b;
+          w_t0 = t0;
+        }
+#pragma unroll
+        for (int qq = 0; qq < QPB; qq++) {
+          const int tq = t0 + qq;
+          if (tq >= nq) break;
+          const int Cq = C - (nq - 1 - tq);  // entries query tq sees
+          float sc = 0.0f;
+#pragma unroll
+          for (int h = 0; h < CSA2_HI; h++)
+            sc = fmaf(wr[qq][h], fmaxf(__uint_as_float(r[qq][h]), 0.0f), sc);
+          if (pos >= Cq) sc = -INFINITY;
+          sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
+          sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
+          sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
+          if ((lane & 7) == 0 && pos < Cq)
+            p.bm[((int64_t)b * nq + tq) * p.bm_stride + pos / CSA2_BLK] = sc;
+        }
+      }
+      if (++acc == ACC) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -233,7 +278,7 @@ __global__ void __launch_bounds__(SC_THREADS, SC_CTAS_PER_SM)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, SC_ACC * SC_N);
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
 }
 
@@ -284,7 +329,8 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
   const int b = blockIdx.y;
   const RescoreJob job = p.job[blockIdx.z];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int C = visible_rows(p.n_rows, b, p.max_rows, p.status);
+  const int C = visible_query(p.n_rows, b, p.nq, p.max_rows, p.status);
+  const int bp = b / p.nq;  // the sequence whose rows the candidates index
   int ncb = p.cand_count[b];
   if (ncb < 0 || ncb > p.cand_stride) {
     set_status(p.status, ST_DEVICE_CHECK);
@@ -332,7 +378,7 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
         int64_t row = -1;
         valid[u][h] = blk >= 0 && pos < C;
         if (valid[u][h]) {
-          row = pos_row(p, b, pos);
+          row = pos_row(p, bp, pos);
           if (row < 0) {
             set_status(p.status, ST_DEVICE_CHECK);
             valid[u][h] = false;
@@ -392,8 +438,8 @@ constexpr int BS_KPT = 16;
 
 __global__ void __launch_bounds__(BS_NT) block_select_kernel(
     const float* __restrict__ bm, int32_t bm_stride, const int32_t* __restrict__ n_rows,
-    int32_t max_rows, int32_t k_req, int32_t* sel, int32_t sel_stride, int32_t* sel_count,
-    uint32_t* status) {
+    int32_t max_rows, int32_t nq, int32_t k_req, int32_t* sel, int32_t sel_stride,
+    int32_t* sel_count, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SelectSmem<BS_NT, BS_KPT>& sm = *reinterpret_cast<SelectSmem<BS_NT, BS_KPT>*>(smem_raw);
   pdl_launch_dependents();
@@ -401,7 +447,7 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int b = blockIdx.y;
-  const int C = visible_rows(n_rows, b, max_rows, status);
+  const int C = visible_query(n_rows, b, nq, max_rows, status);
   const int nblk = (C + CSA2_BLK - 1) / CSA2_BLK;
   const int e0 = (rank * BS_NT + threadIdx.x) * BS_KPT;
   uint32_t key[BS_KPT];
@@ -419,21 +465,39 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
 }
 
 // ------------------------------------------------------------ launchers
-cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
-                        int num_sms, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_scan_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SC_SMEM);
+template <int N, int ACC>
+static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& map_q,
+                                 const ScanParams& p, int num_sms, cudaStream_t st) {
+  using Cfg = ScanCfg<N, ACC>;
+  auto kern = score_scan_kernel<N, ACC>;
+  static int per_sm = 0;  // resident CTAs per SM for this instantiation
+  if (per_sm == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, SC_THREADS, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    per_sm = n < SC_CTAS_PER_SM ? n : SC_CTAS_PER_SM;  // TMEM is sized for at most this many
   }
   const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
-  const int64_t slots = (int64_t)SC_CTAS_PER_SM * num_sms;
+  const int64_t slots = (int64_t)per_sm * num_sms;
   const int grid = (int)(total < slots ? total : slots);
   if (grid <= 0) return cudaSuccess;
-  score_scan_kernel<<<grid, SC_THREADS, SC_SMEM, st>>>(map_k, map_q, p);
+  kern<<<grid, SC_THREADS, Cfg::SMEM, st>>>(map_k, map_q, p);
   return cudaGetLastError();
+}
+
+// Query box rows the scan loads per stage for nq queries of a sequence.
+int scan_query_rows(int nq) { return nq <= 2 ? 16 : (nq <= 4 ? 32 : 64); }
+
+cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
+                        int num_sms, cudaStream_t st) {
+  if (p.nq < 1 || p.nq > CSA2_MAX_QUERY) return cudaErrorInvalidValue;
+  if (p.nq <= 2) return launch_scan_n<16, 4>(map_k, map_q, p, num_sms, st);
+  if (p.nq <= 4) return launch_scan_n<32, 4>(map_k, map_q, p, num_sms, st);
+  return launch_scan_n<64, 2>(map_k, map_q, p, num_sms, st);
 }
 
 // Candidates per sequence: n_cand_blocks * 8, RS_EPC per CTA of a cluster of
@@ -473,8 +537,9 @@ cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_
 }
 
 cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n_rows,
-                                int max_rows, int batch, int k_req, int32_t* sel, int sel_stride,
-                                int32_t* sel_count, uint32_t* status, cudaStream_t st) {
+                                int max_rows, int batch, int nq, int k_req, int32_t* sel,
+                                int sel_stride, int32_t* sel_count, uint32_t* status,
+                                cudaStream_t st) {
   const int nblk_max = (max_rows + CSA2_BLK - 1) / CSA2_BLK;
   int cs = (nblk_max + BS_NT * BS_KPT - 1) / (BS_NT * BS_KPT);
   if (cs < 1) cs = 1;
@@ -504,8 +569,8 @@ cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n
   cfg.attrs = at;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, block_select_kernel, bm, (int32_t)bm_stride, n_rows,
-                            (int32_t)max_rows, (int32_t)k_req, sel, (int32_t)sel_stride,
-                            sel_count, status);
+                            (int32_t)max_rows, (int32_t)nq, (int32_t)k_req, sel,
+                            (int32_t)sel_stride, sel_count, status);
 }
 
 }  // namespace csa2

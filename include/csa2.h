@@ -50,7 +50,8 @@ enum {
   CSA2_W = 128,          /* sliding-window rows [REL §CED; YOM §一]            */
   CSA2_MAX_TOPK = 512,   /* Top-512 [REL §CSA2; YOM §二 table]                 */
   CSA2_MAX_POOL = 2048,  /* 2,048 blocks = 16,384 positions [YOM §二 HSI]      */
-  CSA2_MAX_ROWS = 1 << 20 /* visible entries per sequence (1M context)        */
+  CSA2_MAX_ROWS = 1 << 20, /* visible entries per sequence (1M context)       */
+  CSA2_MAX_QUERY = 8       /* draft positions verified per sequence per step   */
 };
 
 typedef enum {
@@ -299,6 +300,21 @@ csa2_status csa2_sparse_attn_decode(const uint16_t *q, const csa2_kv_view *kv,
  * and pool_count [batch] of the last FULL layer (may be NULL when
  * pool_blocks == 0), out bf16 [L][batch][16][512].
  * modes points to HOST memory; everything else is device memory.
+ *
+ * Multi-query step (n_query = Q in [2, CSA2_MAX_QUERY]): verification of Q
+ * draft positions per sequence whose entries are already in the caches (the
+ * release note and the cnblogs article describe DSpark drafting several
+ * positions that the main model verifies in one pass).  Query t of sequence
+ * b sees the first kv.n_rows[b] - (Q-1-t) global entries and the window rows
+ * [max(0, e_t - 128), e_t) with e_t = swa_len[b] - (Q-1-t).  Every per-query
+ * array gains a query axis after the batch axis, so "batch" above reads
+ * batch x Q: q_idx [L][batch][Q][8][64], w [L][batch][Q][8],
+ * q [L][batch][Q][16][512], idx [L][batch][Q][top_k], idx_count
+ * [L][batch][Q], pool [batch][Q][pool_blocks], pool_count [batch][Q],
+ * out [L][batch][Q][16][512]; the window is swa [L][batch][128 + Q - 1][512]
+ * with swa_len [batch] <= 128 + Q - 1.  The scan reads every indexer-K row
+ * once for all Q queries (one MMA of N = 8Q, padded to 16/32/64).
+ * batch x Q must not exceed 65535.
  */
 typedef struct {
   csa2_kv_view kv;
@@ -317,6 +333,7 @@ typedef struct {
   int32_t *pool;
   int32_t *pool_count;
   uint16_t *out;
+  int32_t n_query; /* queries (draft positions) per sequence; 0 or 1 = one */
 } csa2_group_desc;
 
 size_t csa2_group_workspace_size(const csa2_group_desc *desc);
