@@ -246,6 +246,43 @@ def time_cache_append(csa2, wl, dev, stream, K, W):
             "timing": f"{K} back-to-back calls after {W} warm-up calls, CUDA events"}
 
 
+def time_multi_query(csa2, wl, kv, dev, stream, flush_l2, K, W, Q=4):
+    """Verification of Q draft positions per sequence in one step over the
+    workload's cache (the last Q entries are the drafts), timed like the
+    headline step (L2 flushed between steps, events around each step)."""
+    import torch
+    B, L = wl.B, wl.L
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed + 1)
+    bf = lambda *shape: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16).view(  # noqa: E731
+        torch.int16)
+    q_idx, q = bf(L, B * Q, 8, 64), bf(L, B * Q, 16, 512)
+    w = torch.rand((L, B * Q, 8), generator=g, device=dev)
+    swa = torch.randn((L, B, 128 + Q - 1, 512), generator=g, device=dev).to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    swa_len = torch.full((B,), 128 + Q - 1, dtype=torch.int32, device=dev)
+    grp = csa2.LayerGroup(kv, wl.modes, q_idx, w, q, swa, swa_len, top_k=wl.top_k,
+                          pool_blocks=wl.pool_blocks, n_query=Q)
+    ws = csa2.workspace(grp.workspace_size(), device=dev)
+    for _ in range(W):
+        csa2.csa2_layer_group(grp, ws)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush_l2()
+        ev[i][0].record(stream)
+        csa2.csa2_layer_group(grp, ws)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    csa2.csa2_sync_status(ws)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    return {"queries_per_sequence": Q, "ms_per_step": ms,
+            "value": B * Q * L / (ms * 1e-3), "unit": "query-layer-steps/s",
+            "steps": K, "warmup": W,
+            "note": "indexer K read once per step for all queries (MMA N = 8Q)"}
+
+
 def run_gpu(args, wl, rank, world):
     import torch
 
@@ -379,6 +416,7 @@ def run_gpu(args, wl, rank, world):
     t_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / K, dist, dev)
 
     append = time_cache_append(csa2, wl, dev, stream, K, args.warmup)
+    multi = time_multi_query(csa2, wl, kv, dev, stream, flush_l2, max(10, K // 4), args.warmup)
 
     units = wl.B * wl.L
     value = job_throughput(units, world, t_step)
@@ -408,7 +446,7 @@ def run_gpu(args, wl, rank, world):
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(units, world, t_e2e), "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-            "next_rows": {"cache_append": append},
+            "next_rows": {"cache_append": append, "multi_query": multi},
             "gpu_launches": int(launches * K),
             "gpu_launches_per_step": int(launches),
             "clocks": sampler.summary(),

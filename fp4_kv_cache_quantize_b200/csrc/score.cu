@@ -92,7 +92,9 @@ __device__ __forceinline__ int32_t box_row(const ScanParams& p, int b, int pos0)
   return (int32_t)row;
 }
 
-template <int N, int ACC>
+// ONE: the single-query specialisation (weights held in registers, one TMEM
+// load per tile).
+template <int N, int ACC, bool ONE>
 __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
     score_scan_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_q, const ScanParams p) {
@@ -207,10 +209,10 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
   } else {  // ------------------------------------------ epilogue, 4 warps
     // Thread = one TMEM lane = one position of the tile.  Query tq's score
     // is the weighted ReLU sum over accumulator columns [8 tq, 8 tq + 8).
-    constexpr int QPB = N / 8 < 4 ? N / 8 : 4;  // queries per batch of TMEM loads
+    constexpr int QPB = ONE ? 1 : (N / 8 < 4 ? N / 8 : 4);  // queries per batch of TMEM loads
     const int quarter = warp & 3;  // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
-    const int nq = p.nq;
+    const int nq = ONE ? 1 : p.nq;
     int acc = 0;
     uint32_t acc_phase = 0;
     int cur_b = -1, C = 0, w_b = -1, w_t0 = -1;
@@ -465,21 +467,34 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
 }
 
 // ------------------------------------------------------------ launchers
-template <int N, int ACC>
+template <int N, int ACC, bool ONE>
 static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& map_q,
                                  const ScanParams& p, int num_sms, cudaStream_t st) {
   using Cfg = ScanCfg<N, ACC>;
-  auto kern = score_scan_kernel<N, ACC>;
+  auto kern = score_scan_kernel<N, ACC, ONE>;
   static int per_sm = 0;  // resident CTAs per SM for this instantiation
   if (per_sm == 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, SC_THREADS, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
+    // Resident CTAs per SM from the shared memory, registers and TMEM each
+    // one takes (the runtime's occupancy calculator reports 1 for kernels
+    // that allocate tensor memory, so the limits are applied here).
+    int dev = 0, smem_sm = 0, reserved = 0, regs_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    const int warp_regs = (fa.numRegs * 32 + 255) / 256 * 256;
+    int n = smem_sm / ((int)Cfg::SMEM + reserved);
+    const int by_regs = regs_sm / (warp_regs * (SC_THREADS / 32));
+    const int by_tmem = 512 / (int)Cfg::TMEM_COLS;
+    n = n < by_regs ? n : by_regs;
+    n = n < by_tmem ? n : by_tmem;
     if (n < 1) return cudaErrorInvalidConfiguration;
-    per_sm = n < SC_CTAS_PER_SM ? n : SC_CTAS_PER_SM;  // TMEM is sized for at most this many
+    per_sm = n < SC_CTAS_PER_SM ? n : SC_CTAS_PER_SM;
   }
   const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
   const int64_t slots = (int64_t)per_sm * num_sms;
@@ -495,9 +510,10 @@ int scan_query_rows(int nq) { return nq <= 2 ? 16 : (nq <= 4 ? 32 : 64); }
 cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
                         int num_sms, cudaStream_t st) {
   if (p.nq < 1 || p.nq > CSA2_MAX_QUERY) return cudaErrorInvalidValue;
-  if (p.nq <= 2) return launch_scan_n<16, 4>(map_k, map_q, p, num_sms, st);
-  if (p.nq <= 4) return launch_scan_n<32, 4>(map_k, map_q, p, num_sms, st);
-  return launch_scan_n<64, 2>(map_k, map_q, p, num_sms, st);
+  if (p.nq == 1) return launch_scan_n<16, 4, true>(map_k, map_q, p, num_sms, st);
+  if (p.nq <= 2) return launch_scan_n<16, 4, false>(map_k, map_q, p, num_sms, st);
+  if (p.nq <= 4) return launch_scan_n<32, 4, false>(map_k, map_q, p, num_sms, st);
+  return launch_scan_n<64, 2, false>(map_k, map_q, p, num_sms, st);
 }
 
 // Candidates per sequence: n_cand_blocks * 8, RS_EPC per CTA of a cluster of
