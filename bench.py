@@ -201,25 +201,27 @@ def config_dict(wl):
 
 
 # ------------------------------------------------------------ GPU arm
-def time_cache_append(csa2, wl, dev, stream, K, W):
+def time_cache_append(csa2, wl, dev, stream, K, W, with_cpu):
     """The cache-append step that precedes a decode step (one new main-KV
     entry per sequence, one window entry per layer and sequence), timed with
     events over K back-to-back calls into a scratch cache of the workload's
-    batch and layer count.  Latency-bound: it moves ~100 KB per call."""
+    batch and layer count.  Latency-bound: it moves ~100 KB per call.  The
+    oracle's append is timed on the same inputs (host copies)."""
     import torch
+    from fp4_kv_cache_quantize_b200 import synth
     B, L = wl.B, wl.L
     cap = 64 * ((W + K + 63) // 64 + 1)
-    g = torch.Generator(device=dev)
-    g.manual_seed(wl.seed)
+    rng = synth.rng(wl.seed, 200)
+    x_np = synth.to_bf16_bits(rng.standard_normal((B, 512)).astype(np.float32))
+    w_np = synth.to_bf16_bits((rng.standard_normal((512, 64)) / 512 ** 0.5).astype(np.float32))
+    xs_np = synth.to_bf16_bits(rng.standard_normal((L, B, 512)).astype(np.float32))
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)  # noqa: E731
     codes = torch.zeros((B * cap, 256), dtype=torch.uint8, device=dev)
     scales = torch.zeros((B * cap, 32), dtype=torch.uint8, device=dev)
     idxk = torch.zeros((B * cap, 64), dtype=torch.int16, device=dev)
     n_rows = torch.zeros(B, dtype=torch.int32, device=dev)
     kv = csa2.KVCache(codes, scales, idxk, n_rows, max_rows=cap, seq_stride=cap)
-    x = torch.randn((B, 512), generator=g, device=dev).to(torch.bfloat16).view(torch.int16)
-    w_idx = (torch.randn((512, 64), generator=g, device=dev) / 512 ** 0.5).to(
-        torch.bfloat16).view(torch.int16)
-    x_swa = torch.randn((L, B, 512), generator=g, device=dev).to(torch.bfloat16).view(torch.int16)
+    x, w_idx, x_swa = to_dev(x_np), to_dev(w_np), to_dev(xs_np)
     swa = torch.zeros((L, B, 128, 512), dtype=torch.uint8, device=dev)
     swa_pos = torch.zeros(B, dtype=torch.int32, device=dev)
     swa_len = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -241,27 +243,81 @@ def time_cache_append(csa2, wl, dev, stream, K, W):
     assert int(n_rows.min()) == W + K and int(swa_pos.min()) == W + K
     us = 1e3 * e0.elapsed_time(e1) / K
     per_seq = 1024 + 256 + 32 + 128 + L * (1024 + 512)
-    return {"us_per_call": us, "launches_per_call": 2, "batch": B, "layers": L,
-            "algorithmic_bytes_per_call": B * per_seq + 512 * 64 * 2,
-            "timing": f"{K} back-to-back calls after {W} warm-up calls, CUDA events"}
+    nbytes = B * per_seq + 512 * 64 * 2
+    peak, peak_kind = measured_peaks()
+    out = {"us_per_call": us, "launches_per_call": 2, "batch": B, "layers": L,
+           "algorithmic_bytes_per_call": nbytes,
+           "roofline": {"bound": "latency", "achieved": nbytes / (us * 1e-6) / 1e9, "peak": peak,
+                        "peak_kind": peak_kind, "unit": "GB/s",
+                        "frac": nbytes / (us * 1e-6) / 1e9 / peak, "traffic": None},
+           "timing": f"{K} back-to-back calls after {W} warm-up calls, CUDA events"}
+    if with_cpu:
+        import oracle
+        dm = oracle.dims()
+        okv = oracle.KV(np.zeros((B * cap, 256), np.uint8), np.zeros((B * cap, 32), np.uint8),
+                        np.zeros((B * cap, 64), np.uint16), seq_stride=cap)
+        on = np.zeros(B, np.int64)
+        oswa = np.zeros((L, B, 128, 512), np.uint8)
+        opos, olen = np.zeros(B, np.int64), np.zeros(B, np.int32)
+        n_calls = 20
+        t0 = time.perf_counter()
+        for _ in range(n_calls):
+            oracle.cache_append(okv, dm, on, x_np, w_np, xs_np, oswa, opos, olen)
+        dt = (time.perf_counter() - t0) / n_calls
+        out["cpu_baseline"] = {"value": dt * 1e6, "unit": "us_per_call", "cores": 1,
+                               "kind": "oracle",
+                               "sample": f"{n_calls} oracle appends of the same inputs"}
+    return out
 
 
-def time_multi_query(csa2, wl, kv, dev, stream, flush_l2, K, W, Q=4):
+def oracle_multi_time(wl, Q, q_idx, w, q, swa, swa_len):
+    """The oracle's multi-query step on this workload (one step), with the
+    main-KV rows it reads quantised as in oracle_step_time."""
+    import oracle
+    dm = oracle.dims()
+    codes = np.zeros((wl.pool_rows, 256), np.uint8)
+    scales = np.zeros((wl.pool_rows, 32), np.uint8)
+    idxk = np.zeros((wl.pool_rows, 64), np.uint16)
+    for r0, _, kc in wl.iter_chunks():
+        idxk[r0:r0 + len(kc)] = kc
+    kv = oracle.KV(codes, scales, idxk, seq_stride=wl.seq_stride, page_table=wl.page_table)
+    args = (kv, dm, wl.n_rows, Q, wl.modes, q_idx, w, q, swa, swa_len)
+    r = oracle.layer_group_multi(*args, top_k=wl.top_k, pool_blocks=wl.pool_blocks)
+    rows = set()
+    for b in range(wl.B):
+        for t in range(Q):
+            for l in range(wl.L):
+                pos = r["idx"][l, b, t, :r["idx_count"][l, b, t]]
+                rows.update(wl.row_of(b, pos).tolist())
+    sel = np.array(sorted(rows), dtype=np.int64)
+    xs, _ = wl.rows(sel)
+    c, sc = oracle.quantize_fp4(xs)
+    kv.codes[sel] = c
+    kv.scales[sel] = sc
+    t0 = time.perf_counter()
+    oracle.layer_group_multi(*args, top_k=wl.top_k, pool_blocks=wl.pool_blocks)
+    return time.perf_counter() - t0
+
+
+def time_multi_query(csa2, wl, kv, dev, stream, flush_l2, K, W, with_cpu, Q=4):
     """Verification of Q draft positions per sequence in one step over the
     workload's cache (the last Q entries are the drafts), timed like the
-    headline step (L2 flushed between steps, events around each step)."""
+    headline step (L2 flushed between steps, events around each step), plus
+    a traced pass for the scan's roofline and the oracle beside it."""
     import torch
+    from fp4_kv_cache_quantize_b200 import synth
     B, L = wl.B, wl.L
-    g = torch.Generator(device=dev)
-    g.manual_seed(wl.seed + 1)
-    bf = lambda *shape: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16).view(  # noqa: E731
-        torch.int16)
-    q_idx, q = bf(L, B * Q, 8, 64), bf(L, B * Q, 16, 512)
-    w = torch.rand((L, B * Q, 8), generator=g, device=dev)
-    swa = torch.randn((L, B, 128 + Q - 1, 512), generator=g, device=dev).to(
-        torch.float8_e4m3fn).view(torch.uint8)
-    swa_len = torch.full((B,), 128 + Q - 1, dtype=torch.int32, device=dev)
-    grp = csa2.LayerGroup(kv, wl.modes, q_idx, w, q, swa, swa_len, top_k=wl.top_k,
+    rng = synth.rng(wl.seed, 300 + Q)
+    bf = lambda *shape: synth.to_bf16_bits(rng.standard_normal(shape).astype(np.float32))  # noqa: E731
+    q_idx_np, q_np = bf(L, B, Q, 8, 64), bf(L, B, Q, 16, 512)
+    w_np = rng.uniform(0, 1, (L, B, Q, 8)).astype(np.float32)
+    swa_np = synth.to_e4m3_bits(rng.standard_normal((L, B, 128 + Q - 1, 512)).astype(np.float32))
+    swa_len_np = np.full(B, 128 + Q - 1, np.int32)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(  # noqa: E731
+        a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+    grp = csa2.LayerGroup(kv, wl.modes, to_dev(q_idx_np.reshape(L, B * Q, 8, 64)),
+                          to_dev(w_np.reshape(L, B * Q, 8)), to_dev(q_np.reshape(L, B * Q, 16, 512)),
+                          to_dev(swa_np), to_dev(swa_len_np), top_k=wl.top_k,
                           pool_blocks=wl.pool_blocks, n_query=Q)
     ws = csa2.workspace(grp.workspace_size(), device=dev)
     for _ in range(W):
@@ -277,10 +333,42 @@ def time_multi_query(csa2, wl, kv, dev, stream, flush_l2, K, W, Q=4):
     torch.cuda.synchronize()
     csa2.csa2_sync_status(ws)
     ms = sum(a.elapsed_time(b) for a, b in ev) / K
-    return {"queries_per_sequence": Q, "ms_per_step": ms,
-            "value": B * Q * L / (ms * 1e-3), "unit": "query-layer-steps/s",
-            "steps": K, "warmup": W,
-            "note": "indexer K read once per step for all queries (MMA N = 8Q)"}
+    # traced pass: the scan's own duration for its roofline
+    n_ev, KT = 32, min(K, 20)
+    tev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev * KT)]
+    for e in tev:
+        e.record(stream)
+    torch.cuda.synchronize()
+    scan_ms = []
+    for i in range(KT):
+        tr = csa2.Trace(tev[i * n_ev:(i + 1) * n_ev])
+        flush_l2()
+        csa2.csa2_trace_set(tr)
+        csa2.csa2_layer_group(grp, ws)
+        csa2.csa2_trace_set(None)
+        torch.cuda.synchronize()
+        names = tr.names()
+        for j in range(len(names) - 1):
+            if names[j] == "scan":
+                scan_ms.append(tr.events[j].elapsed_time(tr.events[j + 1]))
+    scan_bytes = 128 * int(wl.n_rows.sum())
+    peak, peak_kind = measured_peaks()
+    t_scan = sum(scan_ms) / len(scan_ms) * 1e-3
+    out = {"queries_per_sequence": Q, "ms_per_step": ms,
+           "value": B * Q * L / (ms * 1e-3), "unit": "query-layer-steps/s",
+           "steps": K, "warmup": W,
+           "roofline": {"bound": "hbm", "kernel": "score_scan_kernel (N = 8Q)",
+                        "achieved": scan_bytes / t_scan / 1e9, "peak": peak,
+                        "peak_kind": peak_kind, "unit": "GB/s",
+                        "frac": scan_bytes / t_scan / 1e9 / peak, "traffic": None,
+                        "algorithmic_bytes_per_launch": scan_bytes},
+           "note": "indexer K read once per step for all queries (MMA N = 8Q)"}
+    if with_cpu:
+        dt = oracle_multi_time(wl, Q, q_idx_np, w_np, q_np, swa_np, swa_len_np)
+        out["cpu_baseline"] = {"value": B * Q * L / dt, "unit": "query-layer-steps/s",
+                               "cores": 1, "kind": "oracle",
+                               "sample": f"one {Q}-query step of {wl.name} on one host core"}
+    return out
 
 
 def run_gpu(args, wl, rank, world):
@@ -415,8 +503,10 @@ def run_gpu(args, wl, rank, world):
     barrier()
     t_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / K, dist, dev)
 
-    append = time_cache_append(csa2, wl, dev, stream, K, args.warmup)
-    multi = time_multi_query(csa2, wl, kv, dev, stream, flush_l2, max(10, K // 4), args.warmup)
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu
+    append = time_cache_append(csa2, wl, dev, stream, K, args.warmup, with_cpu)
+    multi = time_multi_query(csa2, wl, kv, dev, stream, flush_l2, max(10, K // 4), args.warmup,
+                             with_cpu)
 
     units = wl.B * wl.L
     value = job_throughput(units, world, t_step)
