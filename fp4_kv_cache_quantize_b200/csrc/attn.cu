@@ -175,9 +175,9 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
     __syncthreads();         // previous chunk fully consumed
     if (t < AT_CH) {  // validity of each key, for the logits mask
       int64_t row = -1;
+      const int pos = sparse && k0 + t < p.idx_stride ? __ldg(idx + k0 + t) : -1;
       if (k0 + t < nk) {
         if (sparse) {
-          const int pos = __ldg(idx + k0 + t);
           if (pos >= 0 && pos < C) row = kv_row(p, bp, pos);
           if (row < 0) set_status(p.status, ST_DEVICE_CHECK);
         } else {
@@ -194,11 +194,11 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
 #pragma unroll
       for (int u = 0; u < 8; u++) {
         const int i = t + u * AT_NT, r = i >> 4, cc = i & 15;
+        // the index is read without waiting for the count (in bounds of the
+        // index array either way), so both loads are in flight together
+        const int pos = k0 + r < p.idx_stride ? __ldg(idx + k0 + r) : -1;
         int64_t row = -1;
-        if (k0 + r < nk) {
-          const int pos = __ldg(idx + k0 + r);
-          if (pos >= 0 && pos < C) row = kv_row(p, bp, pos);
-        }
+        if (k0 + r < nk && pos >= 0 && pos < C) row = kv_row(p, bp, pos);
         if (row >= 0) {
           cv[u] = __ldg(reinterpret_cast<const uint4*>(p.codes + row * (CSA2_D / 2)) + cc);
           sv[u] = __ldg(reinterpret_cast<const uint16_t*>(p.scales + row * (CSA2_D / 16)) + cc);
@@ -403,6 +403,14 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
   const int64_t slot0 = ((int64_t)li * p.batch + b) * ns;
   __shared__ float f[16];
   __shared__ float invl;
+  // every split's slice is requested before any is used (one L2 round trip,
+  // overlapping the max/sum reduction below)
+  float4 v[AT_CHUNKS];
+#pragma unroll
+  for (int r = 0; r < AT_CHUNKS; r++)
+    v[r] = r < ns ? *reinterpret_cast<const float4*>(p.part_o + (slot0 + r) * (CSA2_H * CSA2_D) +
+                                                     h * CSA2_D + 4 * t)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
   if (t < 32) {
     float m = -INFINITY, l = 0.f;
     if (t < ns) {
@@ -422,13 +430,13 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
   }
   __syncthreads();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int r = 0; r < ns; r++) {
-    const float4 v = *reinterpret_cast<const float4*>(p.part_o + (slot0 + r) * (CSA2_H * CSA2_D) +
-                                                      h * CSA2_D + 4 * t);
-    acc.x = fmaf(f[r], v.x, acc.x);
-    acc.y = fmaf(f[r], v.y, acc.y);
-    acc.z = fmaf(f[r], v.z, acc.z);
-    acc.w = fmaf(f[r], v.w, acc.w);
+#pragma unroll
+  for (int r = 0; r < AT_CHUNKS; r++) {
+    if (r >= ns) break;
+    acc.x = fmaf(f[r], v[r].x, acc.x);
+    acc.y = fmaf(f[r], v[r].y, acc.y);
+    acc.z = fmaf(f[r], v[r].z, acc.z);
+    acc.w = fmaf(f[r], v[r].w, acc.w);
   }
   uint16_t* out = p.layer[li].out + ((int64_t)b * CSA2_H + h) * CSA2_D + 4 * t;
   const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * invl, acc.y * invl);
