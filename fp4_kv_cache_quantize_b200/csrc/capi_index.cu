@@ -147,6 +147,9 @@ static ScanParams scan_params(const csa2_kv_view* kv, const float* w, const Inde
   p.batch = kv->batch;
   p.tiles_per_seq = (kv->max_rows + SC_TILE - 1) / SC_TILE;
   p.nq = nq;
+  p.q_first = 0;
+  p.nq_pass = nq;
+  p.tail = 0;
   p.status = ws.status;
   return p;
 }
@@ -178,10 +181,22 @@ static csa2_status run_scan_select(const csa2_kv_view* kv, const uint16_t* q_idx
   CUtensorMap map_k, map_q;
   csa2_status r = map_rows64(&map_k, kv->idx_k, (uint64_t)kv->pool_rows, 64);
   if (r) return r;
-  r = map_rows64(&map_q, q_idx, (uint64_t)kv->batch * nq * CSA2_HI, scan_query_rows(nq));
-  if (r) return r;
-  trace_mark("scan", st);
-  CSA2_CUDA(launch_scan(map_k, map_q, scan_params(kv, w, ws, nq), num_sms(), st));
+  // one scan launch per pass of up to CSA2_SCAN_QUERIES queries: each reads
+  // the indexer K once and scores that many queries per row
+  ScanParams sp = scan_params(kv, w, ws, nq);
+  int box_rows = 0;
+  for (int q0 = 0; q0 < nq; q0 += CSA2_SCAN_QUERIES) {
+    sp.q_first = q0;
+    sp.nq_pass = nq - q0 < CSA2_SCAN_QUERIES ? nq - q0 : CSA2_SCAN_QUERIES;
+    sp.tail = nq - (q0 + sp.nq_pass);
+    if (scan_query_rows(sp.nq_pass) != box_rows) {
+      box_rows = scan_query_rows(sp.nq_pass);
+      r = map_rows64(&map_q, q_idx, (uint64_t)kv->batch * nq * CSA2_HI, box_rows);
+      if (r) return r;
+    }
+    trace_mark("scan", st);
+    CSA2_CUDA(launch_scan(map_k, map_q, sp, num_sms(), st));
+  }
   trace_mark("block_select", st);
   CSA2_CUDA(launch_block_select(ws.bm, ws.bm_stride, kv->n_rows, kv->max_rows, kv->batch * nq, nq,
                                 P, sel, sel_stride, sel_count, ws.status, st));

@@ -25,9 +25,13 @@ struct ScanParams {
   int32_t batch;
   int32_t tiles_per_seq;
   int32_t nq;        // queries per sequence; w and bm are [batch * nq][...]
+  int32_t q_first;   // this launch scores queries [q_first, q_first + nq_pass)
+  int32_t nq_pass;   // 1..8
+  int32_t tail;      // nq - (q_first + nq_pass): later queries not in this launch
   uint32_t* status;
 };
 constexpr int SC_TILE = 128;
+constexpr int CSA2_SCAN_QUERIES = 8;  // queries one scan launch scores (MMA N <= 64)
 
 constexpr int RS_MAX_JOBS = 8;
 struct RescoreJob {

@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           C = visible_rows(p.n_rows, b, p.max_rows, p.status);
           cur_b = b;
         }
-        if (t * SC_TILE >= C) continue;
+        if (t * SC_TILE >= C - p.tail) continue;
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort)) {
           s.abort = 1;
           set_status(p.status, ST_TIMEOUT);
@@ -150,11 +150,11 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
         }
         const int pos0 = t * SC_TILE;
         const int32_t y0 = box_row(p, b, pos0);
-        const int32_t y1 = pos0 + SC_BOX < C ? box_row(p, b, pos0 + SC_BOX) : y0;
+        const int32_t y1 = pos0 + SC_BOX < C - p.tail ? box_row(p, b, pos0 + SC_BOX) : y0;
         mbar_arrive_expect_tx(&s.full[stage], SC_A_BYTES + Cfg::B_BYTES);
         tma_load_2d(s.a[stage], &map_k, &s.full[stage], 0, y0);
         tma_load_2d(s.a[stage] + SC_BOX * 128, &map_k, &s.full[stage], 0, y1);
-        tma_load_2d(s.b[stage], &map_q, &s.full[stage], 0, b * CSA2_HI * p.nq);
+        tma_load_2d(s.b[stage], &map_q, &s.full[stage], 0, (b * p.nq + p.q_first) * CSA2_HI);
         issued |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == SC_STAGES) {
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
           cur_b = b;
         }
-        if (t * SC_TILE >= C) continue;
+        if (t * SC_TILE >= C - p.tail) continue;
         if (!mbar_wait(&s.full[stage], phase, abort) ||
             !mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort)) {
           s.abort = 1;
@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
     constexpr int QPB = ONE ? 1 : (N / 8 < 4 ? N / 8 : 4);  // queries per batch of TMEM loads
     const int quarter = warp & 3;  // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
-    const int nq = ONE ? 1 : p.nq;
+    const int nq = ONE ? 1 : p.nq_pass;  // queries of this launch
+    const int nq_all = p.nq, q_first = p.q_first;
     int acc = 0;
     uint32_t acc_phase = 0;
     int cur_b = -1, C = 0, w_b = -1, w_t0 = -1;
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
         C = visible_rows(p.n_rows, b, p.max_rows, nullptr);  // the last query's view
         cur_b = b;
       }
-      if (t * SC_TILE >= C) continue;
+      if (t * SC_TILE >= C - p.tail) continue;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.tfull[acc], acc_phase, abort));
       if (!ok) {
         s.abort = 1;
@@ -248,8 +249,9 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           for (int qq = 0; qq < QPB; qq++)
 #pragma unroll
             for (int h = 0; h < CSA2_HI; h++)
-              wr[qq][h] = t0 + qq < nq ? __ldg(p.w + ((int64_t)b * nq + t0 + qq) * CSA2_HI + h)
-                                       : 0.0f;
+              wr[qq][h] = t0 + qq < nq
+                              ? __ldg(p.w + ((int64_t)b * nq_all + q_first + t0 + qq) * CSA2_HI + h)
+                              : 0.0f;
           w_b = b;
           w_t0 = t0;
         }
@@ -257,7 +259,8 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
         for (int qq = 0; qq < QPB; qq++) {
           const int tq = t0 + qq;
           if (tq >= nq) break;
-          const int Cq = C - (nq - 1 - tq);  // entries query tq sees
+          const int gq = q_first + tq;            // query index within the sequence
+          const int Cq = C - (nq_all - 1 - gq);  // entries that query sees
           float sc = 0.0f;
 #pragma unroll
           for (int h = 0; h < CSA2_HI; h++)
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
           if ((lane & 7) == 0 && pos < Cq)
-            p.bm[((int64_t)b * nq + tq) * p.bm_stride + pos / CSA2_BLK] = sc;
+            p.bm[((int64_t)b * nq_all + gq) * p.bm_stride + pos / CSA2_BLK] = sc;
         }
       }
       if (++acc == ACC) {
@@ -504,15 +507,17 @@ static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& ma
   return cudaGetLastError();
 }
 
-// Query box rows the scan loads per stage for nq queries of a sequence.
-int scan_query_rows(int nq) { return nq <= 2 ? 16 : (nq <= 4 ? 32 : 64); }
+// Query box rows the scan loads per stage for nq_pass queries of a sequence.
+int scan_query_rows(int nq_pass) { return nq_pass <= 2 ? 16 : (nq_pass <= 4 ? 32 : 64); }
 
 cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
                         int num_sms, cudaStream_t st) {
-  if (p.nq < 1 || p.nq > CSA2_MAX_QUERY) return cudaErrorInvalidValue;
-  if (p.nq == 1) return launch_scan_n<16, 4, true>(map_k, map_q, p, num_sms, st);
-  if (p.nq <= 2) return launch_scan_n<16, 4, false>(map_k, map_q, p, num_sms, st);
-  if (p.nq <= 4) return launch_scan_n<32, 4, false>(map_k, map_q, p, num_sms, st);
+  if (p.nq_pass < 1 || p.nq_pass > CSA2_SCAN_QUERIES || p.q_first < 0 ||
+      p.q_first + p.nq_pass > p.nq || p.tail != p.nq - (p.q_first + p.nq_pass))
+    return cudaErrorInvalidValue;
+  if (p.nq_pass == 1) return launch_scan_n<16, 4, true>(map_k, map_q, p, num_sms, st);
+  if (p.nq_pass <= 2) return launch_scan_n<16, 4, false>(map_k, map_q, p, num_sms, st);
+  if (p.nq_pass <= 4) return launch_scan_n<32, 4, false>(map_k, map_q, p, num_sms, st);
   return launch_scan_n<64, 2, false>(map_k, map_q, p, num_sms, st);
 }
 

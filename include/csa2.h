@@ -51,7 +51,7 @@ enum {
   CSA2_MAX_TOPK = 512,   /* Top-512 [REL §CSA2; YOM §二 table]                 */
   CSA2_MAX_POOL = 2048,  /* 2,048 blocks = 16,384 positions [YOM §二 HSI]      */
   CSA2_MAX_ROWS = 1 << 20, /* visible entries per sequence (1M context)       */
-  CSA2_MAX_QUERY = 8       /* draft positions verified per sequence per step   */
+  CSA2_MAX_QUERY = 1024    /* queries per sequence per step (drafts, prefill)  */
 };
 
 typedef enum {
@@ -301,10 +301,11 @@ csa2_status csa2_sparse_attn_decode(const uint16_t *q, const csa2_kv_view *kv,
  * pool_blocks == 0), out bf16 [L][batch][16][512].
  * modes points to HOST memory; everything else is device memory.
  *
- * Multi-query step (n_query = Q in [2, CSA2_MAX_QUERY]): verification of Q
- * draft positions per sequence whose entries are already in the caches (the
- * release note and the cnblogs article describe DSpark drafting several
- * positions that the main model verifies in one pass).  Query t of sequence
+ * Multi-query step (n_query = Q in [2, CSA2_MAX_QUERY]): Q new positions per
+ * sequence whose entries are already in the caches, each attending causally:
+ * verification of draft positions (the release note and the cnblogs article
+ * describe DSpark drafting several positions that the main model verifies in
+ * one pass; Q <= 8) and chunked prefill (Q new tokens of a prompt).  Query t of sequence
  * b sees the first kv.n_rows[b] - (Q-1-t) global entries and the window rows
  * [max(0, e_t - 128), e_t) with e_t = swa_len[b] - (Q-1-t).  Every per-query
  * array gains a query axis after the batch axis, so "batch" above reads
@@ -313,7 +314,8 @@ csa2_status csa2_sparse_attn_decode(const uint16_t *q, const csa2_kv_view *kv,
  * [L][batch][Q], pool [batch][Q][pool_blocks], pool_count [batch][Q],
  * out [L][batch][Q][16][512]; the window is swa [L][batch][128 + Q - 1][512]
  * with swa_len [batch] <= 128 + Q - 1.  The scan reads every indexer-K row
- * once for all Q queries (one MMA of N = 8Q, padded to 16/32/64).
+ * once per pass of up to 8 queries (one MMA of N = 8 x queries, padded to
+ * 16/32/64), i.e. ceil(Q / 8) times.
  * batch x Q must not exceed 65535.
  */
 typedef struct {

@@ -95,6 +95,8 @@ def run_and_check(lib, orc, n_rows, Q, modes, swa_len, pool_blocks, seed, paged=
     (2, [20000, 9001], [129, 40]),
     (3, [12000, 700], [130, 3]),
     (8, [9000, 2050], [135, 100]),
+    (20, [3000, 10], [147, 5]),     # three scan passes; early queries of b=1 see nothing
+    (64, [2500], [191]),            # chunked prefill: eight scan passes
 ])
 def test_multi_query_group_parity(lib, orc, Q, n_rows, swa_len):
     run_and_check(lib, orc, n_rows, Q, [FULL, REINDEX, REUSE], swa_len, 2048, seed=300 + Q)
@@ -107,7 +109,7 @@ def test_multi_query_paged_without_pool(lib, orc):
 def test_multi_query_rejects_too_many_queries(lib, orc):
     wl = synth.make("mq", seed=5, B=1, n_rows=[100], modes=[FULL])
     dw = DeviceWorkload(lib, wl, orc)
-    Q = 9
+    Q = 1025
     m = mq_inputs(Q, 1, 1, [10], 6)
     grp = lib.LayerGroup(dw.kv, [FULL], dev(m["q_idx"].reshape(1, Q, 8, 64)),
                          dev(m["w"].reshape(1, Q, 8)), dev(m["q"].reshape(1, Q, 16, 512)),
