@@ -30,13 +30,16 @@ def run_group(lib, dw):
     return grp
 
 
-def compare_group(orc, dw, grp, *, check_out=True):
+def compare_group(orc, dw, grp, *, check_out=True, kv=None, ref=None):
+    """kv/ref: the oracle's cache view and its layer-group result when the
+    caller built them (full-size runs); else both come from dw."""
     wl = dw.wl
-    kv = dw.oracle_kv(orc)
+    kv = kv if kv is not None else dw.oracle_kv(orc)
     dm = orc.dims()
-    ref = orc.layer_group(kv, dm, wl.n_rows, wl.modes, wl.q_idx, wl.w_h, wl.q, wl.swa,
-                          wl.swa_len, top_k=wl.top_k, pool_blocks=wl.pool_blocks,
-                          sm_scale=float(np.float32(512 ** -0.5)))
+    if ref is None:
+        ref = orc.layer_group(kv, dm, wl.n_rows, wl.modes, wl.q_idx, wl.w_h, wl.q, wl.swa,
+                              wl.swa_len, top_k=wl.top_k, pool_blocks=wl.pool_blocks,
+                              sm_scale=float(np.float32(512 ** -0.5)))
     idx = grp.idx.cpu().numpy()
     cnt = grp.idx_count.cpu().numpy()
     out = bf16_to_f64(grp.out)
