@@ -455,14 +455,12 @@ int attn_nsplit(int pairs, int num_sms) {
 }
 
 cudaError_t launch_attn(const AttnParams& p, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(AttnSmem));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static PerDeviceOnce attr;
+  cudaError_t ea = attr.run([](int&) {
+    return cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(AttnSmem));
+  });
+  if (ea != cudaSuccess) return ea;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;

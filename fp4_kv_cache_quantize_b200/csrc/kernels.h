@@ -7,7 +7,34 @@
 
 #include "../../include/csa2.h"
 
+#include <mutex>
+
 namespace csa2 {
+
+// Host-side set-up that a launcher does once per device (kernel attributes,
+// resident-CTA counts), thread-safe; devices beyond the table run it every time.
+struct PerDeviceOnce {
+  static constexpr int kMaxDevices = 64;
+  std::once_flag flag[kMaxDevices];
+  cudaError_t err[kMaxDevices] = {};
+  int value[kMaxDevices] = {};
+  template <class F>  // F: cudaError_t (int& value)
+  cudaError_t run(F f, int* out = nullptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) {
+      int v = 0;
+      e = f(v);
+      if (out) *out = v;
+      return e;
+    }
+    std::call_once(flag[dev], [&] { err[dev] = f(value[dev]); });
+    if (out) *out = value[dev];
+    return err[dev];
+  }
+};
+
 
 void trace_mark(const char* stage, cudaStream_t st);  // capi.cu
 

@@ -475,8 +475,9 @@ static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& ma
                                  const ScanParams& p, int num_sms, cudaStream_t st) {
   using Cfg = ScanCfg<N, ACC>;
   auto kern = score_scan_kernel<N, ACC, ONE>;
-  static int per_sm = 0;  // resident CTAs per SM for this instantiation
-  if (per_sm == 0) {
+  static PerDeviceOnce setup;  // resident CTAs per SM for this instantiation
+  int per_sm = 0;
+  cudaError_t es = setup.run([&](int& v) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg::SMEM);
     if (e != cudaSuccess) return e;
@@ -497,8 +498,10 @@ static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& ma
     n = n < by_regs ? n : by_regs;
     n = n < by_tmem ? n : by_tmem;
     if (n < 1) return cudaErrorInvalidConfiguration;
-    per_sm = n < SC_CTAS_PER_SM ? n : SC_CTAS_PER_SM;
-  }
+    v = n < SC_CTAS_PER_SM ? n : SC_CTAS_PER_SM;
+    return cudaSuccess;
+  }, &per_sm);
+  if (es != cudaSuccess) return es;
   const int64_t total = (int64_t)p.batch * p.tiles_per_seq;
   const int64_t slots = (int64_t)per_sm * num_sms;
   const int grid = (int)(total < slots ? total : slots);
@@ -529,17 +532,16 @@ cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_
   int cs = 1;
   while (cs * RS_EPC < ncand) cs <<= 1;
   if (cs > 16) return cudaErrorInvalidValue;
-  static bool attr_done = false;
   const size_t smem = sizeof(RescoreSmem);
-  if (!attr_done) {
+  static PerDeviceOnce attr;
+  cudaError_t ea = attr.run([smem](int&) {
     cudaError_t e = cudaFuncSetAttribute(rescore_select_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(rescore_select_kernel,
-                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+    return cudaFuncSetAttribute(rescore_select_kernel,
+                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  });
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, batch, n_jobs);
   cfg.blockDim = dim3(RS_NT);
@@ -567,14 +569,12 @@ cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n
   int c2 = 1;
   while (c2 < cs) c2 <<= 1;
   if (c2 > 8) return cudaErrorInvalidValue;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(block_select_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(SelectSmem<BS_NT, BS_KPT>));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static PerDeviceOnce attr;
+  cudaError_t ea = attr.run([](int&) {
+    return cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(SelectSmem<BS_NT, BS_KPT>));
+  });
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(c2, batch, 1);
   cfg.blockDim = dim3(BS_NT);
