@@ -50,6 +50,9 @@ struct ScanCfg {
     uint64_t tfull[ACC], tempty[ACC], done;
     uint32_t tmem_base;
     int abort;
+    // N = 64 (two batches of TMEM loads per tile): each epilogue warp's copy
+    // of the launch's query weights, loaded once per sequence
+    float wq[N > 32 ? 4 * CSA2_SCAN_QUERIES * CSA2_HI : 2];
   };
   static constexpr size_t SMEM = sizeof(Smem) + 1024;
 };
@@ -223,6 +226,13 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
       if (b != cur_b) {
         C = visible_rows(p.n_rows, b, p.max_rows, nullptr);  // the last query's view
         cur_b = b;
+        if constexpr (N > 32) {
+          float* wq = s.wq + (warp - 2) * (CSA2_SCAN_QUERIES * CSA2_HI);
+          __syncwarp();
+          for (int i = lane; i < nq * CSA2_HI; i += 32)
+            wq[i] = __ldg(p.w + ((int64_t)b * nq_all + q_first) * CSA2_HI + i);
+          __syncwarp();
+        }
       }
       if (t * SC_TILE >= C - p.tail) continue;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.tfull[acc], acc_phase, abort));
@@ -244,7 +254,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           tc_fence_before();
           mbar_arrive(&s.tempty[acc]);
         }
-        if (b != w_b || t0 != w_t0) {
+        if (N <= 32 && (b != w_b || t0 != w_t0)) {  // one batch: weights stay in registers
 #pragma unroll
           for (int qq = 0; qq < QPB; qq++)
 #pragma unroll
@@ -255,21 +265,29 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           w_b = b;
           w_t0 = t0;
         }
+        // the QPB queries are independent chains: no early exit, so that
+        // they interleave; a query past the launch's last stores nothing
 #pragma unroll
         for (int qq = 0; qq < QPB; qq++) {
           const int tq = t0 + qq;
-          if (tq >= nq) break;
+          const bool live = tq < nq;              // warp-uniform
           const int gq = q_first + tq;            // query index within the sequence
           const int Cq = C - (nq_all - 1 - gq);  // entries that query sees
           float sc = 0.0f;
 #pragma unroll
-          for (int h = 0; h < CSA2_HI; h++)
-            sc = fmaf(wr[qq][h], fmaxf(__uint_as_float(r[qq][h]), 0.0f), sc);
+          for (int h = 0; h < CSA2_HI; h++) {
+            float wh;
+            if constexpr (N > 32)
+              wh = s.wq[(warp - 2) * (CSA2_SCAN_QUERIES * CSA2_HI) + tq * CSA2_HI + h];
+            else
+              wh = wr[qq][h];
+            sc = fmaf(wh, fmaxf(__uint_as_float(r[qq][h]), 0.0f), sc);
+          }
           if (pos >= Cq) sc = -INFINITY;
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 1));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 2));
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
-          if ((lane & 7) == 0 && pos < Cq)
+          if (live && (lane & 7) == 0 && pos < Cq)
             p.bm[((int64_t)b * nq_all + gq) * p.bm_stride + pos / CSA2_BLK] = sc;
         }
       }
