@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(AP_NT) cache_append_kernel(const AppendParams 
   __shared__ float part[32][CSA2_DI + 1];
   const int b = blockIdx.x, t = threadIdx.x;
   pdl_launch_dependents();
+  pdl_wait();  // counters and rows of the previous append (or other writers)
 
   if (blockIdx.y == 0) {
     const int pos = p.n_rows[b];
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(AP_NT) cache_append_kernel(const AppendParams 
 
 // Advances the counters once every write of the step has landed.
 __global__ void __launch_bounds__(AP_NT) append_commit_kernel(const AppendParams p) {
+  pdl_launch_dependents();
   pdl_wait();
   for (int b = threadIdx.x; b < p.batch; b += AP_NT) {
     const int pos = p.n_rows[b];
@@ -148,19 +150,19 @@ __global__ void __launch_bounds__(AP_NT) append_commit_kernel(const AppendParams
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {
   if (p.batch <= 0) return cudaSuccess;
   const int parts = 1 + (p.n_layers + AP_LAYERS_PER_CTA - 1) / AP_LAYERS_PER_CTA;
-  trace_mark("append", st);
-  cache_append_kernel<<<dim3(p.batch, parts), AP_NT, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1);
+  cfg.gridDim = dim3(p.batch, parts);
   cfg.blockDim = dim3(AP_NT);
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
+  trace_mark("append", st);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, cache_append_kernel, p);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(1);
   trace_mark("append_commit", st);
   return cudaLaunchKernelEx(&cfg, append_commit_kernel, p);
 }

@@ -134,6 +134,9 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   volatile int* abort = &s.abort;
+  // The prologue above overlaps the previous kernel (e.g. the cache append
+  // that wrote the newest rows); nothing it wrote is read before this.
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {  // ---------------------------------- TMA producer
@@ -524,8 +527,17 @@ static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& ma
   const int64_t slots = (int64_t)per_sm * num_sms;
   const int grid = (int)(total < slots ? total : slots);
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, SC_THREADS, Cfg::SMEM, st>>>(map_k, map_q, p);
-  return cudaGetLastError();
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(SC_THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map_k, map_q, p);
 }
 
 // Query box rows the scan loads per stage for nq_pass queries of a sequence.
