@@ -92,6 +92,7 @@ _attn = _sig("csa2_sparse_attn_decode", C.c_int,
              [_vp, C.POINTER(KVView), _vp, _vp, _i32, _vp, _vp, C.c_float, _vp, _vp, _sz, _vp])
 _append = _sig("csa2_cache_append", C.c_int,
                 [C.POINTER(KVView), _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_selftest_wait = _sig("csa2_selftest_bounded_wait", C.c_int, [_vp, _sz, _i64, _vp])
 _trace_set = _sig("csa2_trace_set", None, [_vp])
 _group_ws = _sig("csa2_group_workspace_size", _sz, [C.POINTER(GroupDesc)])
 _group = _sig("csa2_layer_group", C.c_int, [C.POINTER(GroupDesc), _vp, _sz, _vp])
@@ -156,6 +157,10 @@ def csa2_workspace_init(ws, stream=None):
 
 def csa2_sync_status(ws, stream=None):
     _check(_sync_status(_ptr(ws), _stream(stream)))
+
+
+def csa2_selftest_bounded_wait(ws, cycles: int, stream=None):
+    _check(_selftest_wait(_ptr(ws), ws.numel(), int(cycles), _stream(stream)))
 
 
 def csa2_quantize_fp4(x_bf16, codes, scales, stream=None):

@@ -36,6 +36,19 @@ csa2_status cuda_fail(cudaError_t e, const char* what) {
   return fail(CSA2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// A wait on an mbarrier that nothing completes, through the same bounded
+// wait every pipeline uses: it gives up after `budget` cycles and records
+// ST_TIMEOUT, then the kernel returns normally.
+__global__ void bounded_wait_selftest_kernel(uint32_t* status, long long budget) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0, nullptr, budget)) set_status(status, ST_TIMEOUT);
+    mbar_arrive(&bar);  // complete the phase so that nothing is left pending
+  }
+}
+
 int num_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -75,6 +88,20 @@ csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, csa2_stream_t stream)
                "workspace of %zu bytes is smaller than its %d-byte header", ws_bytes,
                CSA2_WS_HEADER);
   CSA2_CUDA(cudaMemsetAsync(ws, 0, CSA2_WS_HEADER, (cudaStream_t)stream));
+  return CSA2_OK;
+}
+
+csa2_status csa2_selftest_bounded_wait(void* ws, size_t ws_bytes, int64_t cycles,
+                                       csa2_stream_t stream) {
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE,
+               "workspace of %zu bytes is smaller than its %d-byte header", ws_bytes,
+               CSA2_WS_HEADER);
+  CSA2_REQUIRE(cycles >= 1000 && cycles <= kWaitCycles, CSA2_ERR_INVALID_ARG,
+               "cycles = %lld outside [1000, %lld]", (long long)cycles, (long long)kWaitCycles);
+  bounded_wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(static_cast<uint32_t*>(ws),
+                                                                  (long long)cycles);
+  CSA2_CUDA(cudaGetLastError());
   return CSA2_OK;
 }
 

@@ -150,6 +150,15 @@ csa2_status csa2_cache_append(const csa2_kv_view *kv, const uint16_t *x, const u
                               int32_t *swa_pos, int32_t *swa_len, void *ws, size_t ws_bytes,
                               csa2_stream_t stream);
 
+/* Self-test of the device-side failure path: launches one warp that waits on
+ * a barrier nothing completes, through the same bounded wait every pipeline
+ * wait in this library uses; after `cycles` SM clock cycles (1,000 to
+ * 2,000,000,000) the wait gives up, records the timeout bit in the status
+ * word of ws, and the kernel returns.  The next csa2_sync_status then returns
+ * CSA2_ERR_TIMEOUT and the context stays usable.  Nothing faults or hangs. */
+csa2_status csa2_selftest_bounded_wait(void *ws, size_t ws_bytes, int64_t cycles,
+                                       csa2_stream_t stream);
+
 /* ---------------------------------------------------------------- tracing */
 
 /*
