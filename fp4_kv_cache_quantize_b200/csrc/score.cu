@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
 
 // --------------------------------------------- block Top-k (pool) select
 constexpr int BS_NT = 1024;
-constexpr int BS_KPT = 16;
+constexpr int BS_KPT = 8;   // 131,072 block maxima (1M positions) over a 16-CTA cluster
 
 __global__ void __launch_bounds__(BS_NT) block_select_kernel(
     const float* __restrict__ bm, int32_t bm_stride, const int32_t* __restrict__ n_rows,
@@ -598,11 +598,15 @@ cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n
   if (cs < 1) cs = 1;
   int c2 = 1;
   while (c2 < cs) c2 <<= 1;
-  if (c2 > 8) return cudaErrorInvalidValue;
+  if (c2 > 16) return cudaErrorInvalidValue;
   static PerDeviceOnce attr;
   cudaError_t ea = attr.run([](int&) {
-    return cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sizeof(SelectSmem<BS_NT, BS_KPT>));
+    cudaError_t e = cudaFuncSetAttribute(block_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(SelectSmem<BS_NT, BS_KPT>));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(block_select_kernel,
+                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   });
   if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
