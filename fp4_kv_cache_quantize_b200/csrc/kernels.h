@@ -85,6 +85,7 @@ struct RescoreParams {
   uint32_t* status;
 };
 
+int num_sms();  // SMs of the current device (capi.cu)
 cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, const ScanParams& p,
                         int num_sms, cudaStream_t st);
 cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,

@@ -309,16 +309,15 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
 }
 
 // ------------------------------------------------- rescore + Top-k select
-constexpr int RS_NT = 256;
-constexpr int RS_GB = 4;  // groups of 16 candidates whose loads a warp keeps in flight
+constexpr int RS_GB = 4;      // groups of 16 candidates whose loads a warp keeps in flight
+constexpr int RS_EPC = 1024;  // candidates per CTA (threads x candidates per thread)
 
-
-
-constexpr int RS_KPT = 4;                 // candidates per thread
-constexpr int RS_EPC = RS_NT * RS_KPT;    // candidates per CTA
-
+// Two shapes of the same CTA: 512 threads x 2 candidates when the launch's
+// clusters fit on the GPU at once (shorter scoring and counting chains),
+// 256 x 4 otherwise (twice the CTAs per SM for many (layer, sequence) jobs).
+template <int NT>
 struct RescoreSmem {
-  SelectSmem<RS_NT, RS_KPT> sel;
+  SelectSmem<NT, RS_EPC / NT> sel;
   alignas(16) uint32_t keys[RS_EPC];
   int32_t blocks[RS_EPC / CSA2_BLK];
 };
@@ -344,8 +343,11 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+template <int RS_NT>
 __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescoreParams p) {
   constexpr int EPC = RS_EPC;  // candidates per CTA
+  constexpr int RS_KPT = RS_EPC / RS_NT;
+  using RescoreSmem = csa2::RescoreSmem<RS_NT>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RescoreSmem& s = *reinterpret_cast<RescoreSmem*>(smem_raw);
   pdl_launch_dependents();
@@ -556,25 +558,22 @@ cudaError_t launch_scan(const CUtensorMap& map_k, const CUtensorMap& map_q, cons
 
 // Candidates per sequence: n_cand_blocks * 8, RS_EPC per CTA of a cluster of
 // up to 16 CTAs that scores and selects them together.
-cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
-                           cudaStream_t st) {
-  const int ncand = n_cand_blocks * CSA2_BLK;
-  int cs = 1;
-  while (cs * RS_EPC < ncand) cs <<= 1;
-  if (cs > 16) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(RescoreSmem);
+template <int NT>
+static cudaError_t launch_rescore_nt(const RescoreParams& p, int n_jobs, int batch, int cs,
+                                     cudaStream_t st) {
+  const size_t smem = sizeof(RescoreSmem<NT>);
   static PerDeviceOnce attr;
   cudaError_t ea = attr.run([smem](int&) {
-    cudaError_t e = cudaFuncSetAttribute(rescore_select_kernel,
+    cudaError_t e = cudaFuncSetAttribute(rescore_select_kernel<NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(rescore_select_kernel,
+    return cudaFuncSetAttribute(rescore_select_kernel<NT>,
                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   });
   if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, batch, n_jobs);
-  cfg.blockDim = dim3(RS_NT);
+  cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute at[2];
@@ -586,7 +585,18 @@ cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, rescore_select_kernel, p);
+  return cudaLaunchKernelEx(&cfg, rescore_select_kernel<NT>, p);
+}
+
+cudaError_t launch_rescore(const RescoreParams& p, int n_jobs, int batch, int n_cand_blocks,
+                           cudaStream_t st) {
+  const int ncand = n_cand_blocks * CSA2_BLK;
+  int cs = 1;
+  while (cs * RS_EPC < ncand) cs <<= 1;
+  if (cs > 16) return cudaErrorInvalidValue;
+  const int64_t ctas = (int64_t)cs * batch * n_jobs;
+  if (ctas <= num_sms()) return launch_rescore_nt<512>(p, n_jobs, batch, cs, st);
+  return launch_rescore_nt<256>(p, n_jobs, batch, cs, st);
 }
 
 cudaError_t launch_block_select(const float* bm, int bm_stride, const int32_t* n_rows,
