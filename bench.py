@@ -441,6 +441,34 @@ def run_gpu(args, wl, rank, world):
         step()
     csa2.csa2_sync_status(ws)
 
+    def capture(g_grp):
+        """One decode step as a CUDA graph (its launches keep their
+        programmatic-serialisation edges), or the exception that stopped it."""
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                csa2.csa2_layer_group(g_grp, ws)
+            torch.cuda.synchronize()
+            return graph
+        except Exception as exc:  # noqa: BLE001  (reported, then direct launches)
+            torch.cuda.synchronize()
+            return exc
+
+    ref_idx, ref_out = grp.idx.clone(), grp.out.clone()
+    graph = capture(grp)
+    if isinstance(graph, torch.cuda.CUDAGraph):
+        grp.idx.fill_(-9)
+        graph.replay()
+        torch.cuda.synchronize()
+        csa2.csa2_sync_status(ws)
+        assert torch.equal(grp.idx, ref_idx) and torch.equal(grp.out, ref_out), \
+            "graph replay differs from direct launches"
+        step_launch = "cuda_graph"
+        run_step = graph.replay
+    else:
+        step_launch = f"direct ({type(graph).__name__}: {graph})"[:200]
+        run_step = step
+
     # ---- timed device loop
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -451,7 +479,7 @@ def run_gpu(args, wl, rank, world):
         for i in range(K):
             flush_l2()
             ev[i][0].record(stream)
-            step()
+            run_step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -503,6 +531,14 @@ def run_gpu(args, wl, rank, world):
     grp2 = csa2.LayerGroup(kv, wl.modes, q_idx2, w_h2, q2, swa, swa_len, top_k=wl.top_k,
                            pool_blocks=wl.pool_blocks)
     sets.append((q_idx2, w_h2, q2, grp2))
+    if step_launch == "cuda_graph":
+        csa2.csa2_layer_group(grp2, ws)   # set up outside the capture
+        torch.cuda.synchronize()
+        g2 = capture(grp2)
+        runs = [graph.replay, g2.replay if isinstance(g2, torch.cuda.CUDAGraph) else (
+            lambda: csa2.csa2_layer_group(grp2, ws))]
+    else:
+        runs = [step, lambda: csa2.csa2_layer_group(grp2, ws)]
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     h_outs = [h_out, torch.empty_like(h_out).pin_memory()]
     h_idxs = [h_idx, torch.empty_like(h_idx).pin_memory()]
@@ -526,7 +562,7 @@ def run_gpu(args, wl, rank, world):
             ev_in[j].record(s_in)
         stream.wait_event(ev_in[j])
         stream.wait_event(ev_out[j])             # step i-2's results have left set j
-        csa2.csa2_layer_group(g, ws)
+        runs[j]()
         ev_done[j].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[j])
@@ -573,6 +609,7 @@ def run_gpu(args, wl, rank, world):
             "config": config_dict(wl),
             "hbm_gbs_algorithmic": ab["total"] / (t_step * 1e-3) / 1e9,
             "algorithmic_bytes_per_step": ab["total"],
+            "step_launch": step_launch,
             "stage_us": stage_us_step,
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(units, world, t_e2e), "unit": UNIT,
