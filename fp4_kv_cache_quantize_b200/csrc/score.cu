@@ -31,13 +31,17 @@ constexpr int SC_BOX = 64;                 // rows per TMA box
 constexpr int SC_STAGES = 3;
 constexpr int SC_CTAS_PER_SM = 4;          // up to four independent pipelines per SM
 constexpr int SC_A_BYTES = SC_TILE * 128;  // 16 KB of indexer K per stage
-constexpr int SC_THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr int SC_THREADS = 192;            // producer, MMA, 4 epilogue warps (N <= 32)
 
 // One instantiation per MMA width N: the 8 indexer heads of every query of a
 // sequence (nq queries, 8 nq <= N), padded to 16, 32 or 64; ACC accumulators
 // of N fp32 columns in TMEM.
 template <int N, int ACC>
 struct ScanCfg {
+  // N = 64: 8 epilogue warps, two per TMEM lane quarter, each with half the
+  // queries (the per-row work of 8 queries would otherwise limit the pipeline)
+  static constexpr int EPI_WARPS = N > 32 ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int B_BYTES = N * 128;  // indexer queries per stage
   static constexpr uint32_t IDESC = idesc_bf16_f32(SC_TILE, N);
   static constexpr uint32_t TMEM_COLS = N * ACC;
@@ -52,7 +56,7 @@ struct ScanCfg {
     int abort;
     // N = 64 (two batches of TMEM loads per tile): each epilogue warp's copy
     // of the launch's query weights, loaded once per sequence
-    float wq[N > 32 ? 4 * CSA2_SCAN_QUERIES * CSA2_HI : 2];
+    float wq[N > 32 ? 8 * CSA2_SCAN_QUERIES * CSA2_HI : 2];
   };
   static constexpr size_t SMEM = sizeof(Smem) + 1024;
 };
@@ -98,7 +102,7 @@ __device__ __forceinline__ int32_t box_row(const ScanParams& p, int b, int pos0)
 // ONE: the single-query specialisation (weights held in registers, one TMEM
 // load per tile).
 template <int N, int ACC, bool ONE>
-__global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
+__global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PER_SM : (N <= 32 ? 3 : 2))
     score_scan_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_q, const ScanParams p) {
   using Cfg = ScanCfg<N, ACC>;
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
     }
     for (int i = 0; i < ACC; i++) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], 4 * 32);
+      mbar_init(&s.tempty[i], Cfg::EPI_WARPS * 32);
     }
     mbar_init(&s.done, 1);
     s.abort = 0;
@@ -247,15 +251,20 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * N);
       const int pos = t * SC_TILE + row;
-      for (int t0 = 0; t0 < nq; t0 += QPB) {
+      // this warp's queries: all of them, or its half when 8 warps share a tile
+      const int qlo = Cfg::EPI_WARPS == 8 ? 4 * ((warp - 2) >> 2) : 0;
+      const int qhi = Cfg::EPI_WARPS == 8 ? min(nq, qlo + 4) : nq;
+      bool arrived = false;
+      for (int t0 = qlo; t0 < qhi; t0 += QPB) {
         uint32_t r[QPB][8];
 #pragma unroll
         for (int qq = 0; qq < QPB; qq++)
-          if (t0 + qq < nq) tmem_ld_x8(tbase + (uint32_t)(8 * (t0 + qq)), r[qq]);
+          if (t0 + qq < qhi) tmem_ld_x8(tbase + (uint32_t)(8 * (t0 + qq)), r[qq]);
         tmem_ld_wait();
-        if (t0 + QPB >= nq) {  // every load of this accumulator has completed
+        if (t0 + QPB >= qhi) {  // every load of this warp from the accumulator has completed
           tc_fence_before();
           mbar_arrive(&s.tempty[acc]);
+          if constexpr (Cfg::EPI_WARPS == 8) arrived = true;
         }
         if (N <= 32 && (b != w_b || t0 != w_t0)) {  // one batch: weights stay in registers
 #pragma unroll
@@ -273,7 +282,7 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
 #pragma unroll
         for (int qq = 0; qq < QPB; qq++) {
           const int tq = t0 + qq;
-          const bool live = tq < nq;              // warp-uniform
+          const bool live = tq < qhi;             // warp-uniform
           const int gq = q_first + tq;            // query index within the sequence
           const int Cq = C - (nq_all - 1 - gq);  // entries that query sees
           float sc = 0.0f;
@@ -292,6 +301,12 @@ __global__ void __launch_bounds__(SC_THREADS, N <= 16 ? SC_CTAS_PER_SM : 3)
           sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 4));
           if (live && (lane & 7) == 0 && pos < Cq)
             p.bm[((int64_t)b * nq_all + gq) * p.bm_stride + pos / CSA2_BLK] = sc;
+        }
+      }
+      if constexpr (Cfg::EPI_WARPS == 8) {
+        if (!arrived) {  // a warp with no query of this launch still releases the tile
+          tc_fence_before();
+          mbar_arrive(&s.tempty[acc]);
         }
       }
       if (++acc == ACC) {
@@ -516,7 +531,7 @@ static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& ma
     if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
     const int warp_regs = (fa.numRegs * 32 + 255) / 256 * 256;
     int n = smem_sm / ((int)Cfg::SMEM + reserved);
-    const int by_regs = regs_sm / (warp_regs * (SC_THREADS / 32));
+    const int by_regs = regs_sm / (warp_regs * (Cfg::THREADS / 32));
     const int by_tmem = 512 / (int)Cfg::TMEM_COLS;
     n = n < by_regs ? n : by_regs;
     n = n < by_tmem ? n : by_tmem;
@@ -534,7 +549,7 @@ static cudaError_t launch_scan_n(const CUtensorMap& map_k, const CUtensorMap& ma
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(SC_THREADS);
+  cfg.blockDim = dim3(Cfg::THREADS);
   cfg.dynamicSmemBytes = Cfg::SMEM;
   cfg.stream = st;
   cfg.attrs = at;
