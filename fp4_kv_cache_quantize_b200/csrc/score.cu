@@ -31,7 +31,6 @@ constexpr int SC_BOX = 64;                 // rows per TMA box
 constexpr int SC_STAGES = 3;
 constexpr int SC_CTAS_PER_SM = 4;          // up to four independent pipelines per SM
 constexpr int SC_A_BYTES = SC_TILE * 128;  // 16 KB of indexer K per stage
-constexpr int SC_THREADS = 192;            // producer, MMA, 4 epilogue warps (N <= 32)
 
 // One instantiation per MMA width N: the 8 indexer heads of every query of a
 // sequence (nq queries, 8 nq <= N), padded to 16, 32 or 64; ACC accumulators
