@@ -18,7 +18,9 @@
 // (coalesced, to the workspace, where they stay in L2) and attn_merge_kernel,
 // one CTA per (layer, sequence, head), combines them with log-sum-exp
 // weights.  Each thread derives its gather addresses from the indices
-// directly, and the query load overlaps the first gather.
+// directly, and the query load overlaps the first gather.  With several
+// queries per sequence, blockIdx.y runs over sequences x queries: each query
+// sees the entries and the window rows up to its own position.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>

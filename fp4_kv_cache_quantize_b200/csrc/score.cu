@@ -8,16 +8,20 @@
 //    into a 3-stage shared-memory ring (128B-swizzled tiles of 128 positions),
 //    four CTAs per SM (four independent producer/MMA/epilogue pipelines keep
 //    more requests in flight than one deep ring per CTA does),
-//    one thread issues tcgen05.mma (M = 128 positions, N = 16 >= 8 indexer
-//    heads, K = 64) into a double-buffered TMEM accumulator, and four
-//    epilogue warps read the dot products back (tcgen05.ld), apply
-//    s = sum_h w_h * relu(q_h . k), and write only the block maxima of
-//    8-position blocks.  Scores themselves never touch HBM.
+//    one thread issues tcgen05.mma (M = 128 positions, N = 8 indexer heads
+//    per query padded to 16/32/64, K = 64) into a ring of TMEM accumulators,
+//    and four (eight for N = 64) epilogue warps read the dot products back
+//    (tcgen05.ld), apply s = sum_h w_h * relu(q_h . k) per query, and write
+//    only the block maxima of 8-position blocks.  Scores never touch HBM.
+//    With several queries per sequence (draft verification, chunked
+//    prefill) one launch scores up to 8 of them per indexer-K row.
 //  * rescore_select_kernel: scores the positions of a set of candidate blocks
 //    (the HSI pool for Reindex layers, the Full layer's top blocks for its own
-//    Top-512) with legacy mma.sync tensor-core tiles over gathered rows, then
+//    Top-512) with mma.sync tensor-core tiles over gathered rows, then
 //    selects the exact Top-k in the same cluster with the radix select of
 //    select.cuh.  Several (layer, sequence) jobs run in one launch.
+//  * block_select_kernel: the HSI pool, the top blocks by block maximum, with
+//    the same radix select over a cluster of up to 16 CTAs per sequence.
 #include <cuda_bf16.h>
 
 #include "csa2_internal.cuh"
