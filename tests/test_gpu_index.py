@@ -204,6 +204,35 @@ def test_attention_device_check_on_bad_index(lib, orc):
     lib.csa2_sync_status(ws)  # cleared
 
 
+def test_index_device_check_on_bad_page(lib, orc):
+    """A page-table entry outside the row pool is never dereferenced by the
+    scan (its TMA box is read as zeros), the rescore or the attention: the
+    affected rows are skipped and csa2_sync_status reports
+    CSA2_ERR_DEVICE_CHECK; the rest of the step still runs."""
+    wl = synth.make("bp", seed=12, B=2, n_rows=[3000, 900], modes=[FULL], paged=True)
+    dw = DeviceWorkload(lib, wl, orc)
+    pt = wl.page_table.copy()
+    pt[0, 5] = 10 ** 6          # page 5 of sequence 0: far outside the pool
+    pt[1, 2] = -3               # a negative page id
+    kv = lib.KVCache(dw.codes, dw.scales, dw.idxk, dw.n_rows, max_rows=int(wl.n_rows.max()),
+                     page_table=dev(pt))
+    idx = torch.full((2, 512), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((2,), -7, dtype=torch.int32, device="cuda")
+    pool = torch.full((2, 2048), -7, dtype=torch.int32, device="cuda")
+    pcnt = torch.full((2,), -7, dtype=torch.int32, device="cuda")
+    ws = lib.workspace(lib.csa2_index_workspace_size(kv, 512, 2048))
+    lib.csa2_index_full(kv, dw.q_idx[0], dw.w[0], 512, 2048, idx, cnt, pool, pcnt, ws)
+    with pytest.raises(lib.Csa2Error) as e:
+        lib.csa2_sync_status(ws)
+    assert e.value.status == 7
+    cnt = cnt.cpu().numpy()
+    assert cnt[0] == 512 and cnt[1] == 512
+    i0 = idx.cpu().numpy()
+    assert not np.isin(i0[0], np.arange(5 * 64, 6 * 64)).any()   # nothing from the bad page
+    assert not np.isin(i0[1], np.arange(2 * 64, 3 * 64)).any()
+    lib.csa2_sync_status(ws)  # cleared
+
+
 def test_host_side_argument_errors(lib, orc):
     wl = synth.make("at", seed=4, B=1, n_rows=[100], modes=[FULL])
     dw = DeviceWorkload(lib, wl, orc)
