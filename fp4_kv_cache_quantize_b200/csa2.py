@@ -98,6 +98,31 @@ _group_ws = _sig("csa2_group_workspace_size", _sz, [C.POINTER(GroupDesc)])
 _group = _sig("csa2_layer_group", C.c_int, [C.POINTER(GroupDesc), _vp, _sz, _vp])
 
 
+class CpShard(C.Structure):
+    _fields_ = [("rank", C.c_int32), ("world", C.c_int32), ("shard_rows", C.c_int32)]
+
+
+_PS = C.POINTER(CpShard)
+_cp_ws = _sig("csa2_cp_workspace_size", _sz, [_PS, _i32, _i32, _i32])
+_cp_partial_floats = _sig("csa2_cp_partial_floats", _sz, [_i32, _i32])
+_cp_local_rows = _sig("csa2_cp_local_rows", C.c_int, [_PS, _vp, _i32, _vp, _vp, _sz, _vp])
+_cp_block_max = _sig("csa2_cp_block_max", C.c_int,
+                     [_PS, C.POINTER(KVView), _vp, _vp, _vp, _vp, _sz, _vp])
+_cp_pool = _sig("csa2_cp_pool", C.c_int, [_PS, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _sz, _vp])
+_cp_filter = _sig("csa2_cp_filter", C.c_int,
+                  [_PS, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp])
+_cp_select_local = _sig("csa2_cp_select_local", C.c_int,
+                        [_PS, C.POINTER(KVView), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _sz,
+                         _vp])
+_cp_select_merge = _sig("csa2_cp_select_merge", C.c_int,
+                        [_PS, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp])
+_cp_attn_partial = _sig("csa2_cp_attn_partial", C.c_int,
+                        [_PS, C.POINTER(KVView), _i32, _vp, _vp, _vp, _vp, _vp, _i32, C.c_float,
+                         _vp, _vp, _sz, _vp])
+_cp_attn_combine = _sig("csa2_cp_attn_combine", C.c_int,
+                        [_PS, _vp, _i32, _i32, _vp, _vp, _sz, _vp])
+
+
 def _check(rc: int):
     if rc != 0:
         raise Csa2Error(rc, _last_error().decode())
@@ -286,3 +311,64 @@ class Trace:
 
 def csa2_trace_set(trace):
     _trace_set(C.addressof(trace.s) if trace is not None else None)
+
+
+# ------------------------------------------------- context-parallel decode
+def csa2_cp_workspace_size(shard: CpShard, batch: int, n_layers: int, top_k: int) -> int:
+    return _cp_ws(C.byref(shard), batch, n_layers, top_k)
+
+
+def csa2_cp_partial_floats(batch: int, n_layers: int) -> int:
+    return _cp_partial_floats(batch, n_layers)
+
+
+def csa2_cp_local_rows(shard: CpShard, n_rows, local_rows, ws, stream=None):
+    _check(_cp_local_rows(C.byref(shard), _ptr(n_rows), int(n_rows.numel()), _ptr(local_rows),
+                          _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_cp_block_max(shard: CpShard, kv: KVCache, q_idx, w, bm, ws, stream=None):
+    _check(_cp_block_max(C.byref(shard), C.byref(kv.view), _ptr(q_idx), _ptr(w), _ptr(bm),
+                         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_cp_pool(shard: CpShard, bm_all, n_rows, P, pool, pool_count, ws, stream=None):
+    _check(_cp_pool(C.byref(shard), _ptr(bm_all), _ptr(n_rows), int(n_rows.numel()), P,
+                    _ptr(pool), _ptr(pool_count), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_cp_filter(shard: CpShard, unit, lst, count, out, out_count, ws, copy=None,
+                   copy_count=None, stream=None):
+    """lst int32 [batch][stride] -> out int32 [batch][out_stride] (see csa2.h)."""
+    _check(_cp_filter(C.byref(shard), unit, _ptr(lst), _ptr(count), int(lst.shape[-1]),
+                      int(count.numel()), _ptr(out), _ptr(out_count), int(out.shape[-1]),
+                      _ptr(copy), _ptr(copy_count), _ptr(ws), ws.numel(),
+                      _stream(stream)))
+
+
+def csa2_cp_select_local(shard: CpShard, kv: KVCache, q_idx, w, cand, cand_count, top_k, send,
+                         ws, stream=None):
+    _check(_cp_select_local(C.byref(shard), C.byref(kv.view), _ptr(q_idx), _ptr(w),
+                            _ptr(cand), _ptr(cand_count), int(cand.shape[-1]), top_k,
+                            _ptr(send), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_cp_select_merge(shard: CpShard, gathered, n_jobs, job, batch, top_k, idx, idx_count,
+                         ws, stream=None):
+    _check(_cp_select_merge(C.byref(shard), _ptr(gathered), n_jobs, job, batch, top_k,
+                            _ptr(idx), _ptr(idx_count), _ptr(ws), ws.numel(),
+                            _stream(stream)))
+
+
+def csa2_cp_attn_partial(shard: CpShard, kv: KVCache, q, swa, swa_len, idx_local, idx_count,
+                         sm_scale, partial, ws, stream=None):
+    L = int(q.shape[0])
+    _check(_cp_attn_partial(C.byref(shard), C.byref(kv.view), L, _ptr(q), _ptr(swa),
+                            _ptr(swa_len), _ptr(idx_local), _ptr(idx_count),
+                            int(idx_local.shape[-1]), float(sm_scale), _ptr(partial), _ptr(ws),
+                            ws.numel(), _stream(stream)))
+
+
+def csa2_cp_attn_combine(shard: CpShard, gathered, n_layers, batch, out, ws, stream=None):
+    _check(_cp_attn_combine(C.byref(shard), _ptr(gathered), n_layers, batch, _ptr(out),
+                            _ptr(ws), ws.numel(), _stream(stream)))

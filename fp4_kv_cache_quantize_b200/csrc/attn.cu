@@ -456,7 +456,7 @@ int attn_nsplit(int pairs, int num_sms) {
   return 10;
 }
 
-cudaError_t launch_attn(const AttnParams& p, cudaStream_t st) {
+cudaError_t launch_attn(const AttnParams& p, cudaStream_t st, bool merge) {
   static PerDeviceOnce attr;
   cudaError_t ea = attr.run([](int&) {
     return cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -475,7 +475,7 @@ cudaError_t launch_attn(const AttnParams& p, cudaStream_t st) {
   cfg.numAttrs = 1;
   trace_mark("attn", st);
   cudaError_t e = cudaLaunchKernelEx(&cfg, attn_decode_kernel, p);
-  if (e != cudaSuccess || p.nsplit == 1) return e;
+  if (e != cudaSuccess || p.nsplit == 1 || !merge) return e;
   cudaLaunchConfig_t mc = {};
   mc.gridDim = dim3(CSA2_H, p.batch, p.n_layers);
   mc.blockDim = dim3(128);

@@ -231,6 +231,72 @@ static GroupWs group_ws_layout(const csa2_group_desc* d, uint8_t* base) {
   return g;
 }
 
+// ------------------------------------------------- context-parallel decode
+#define CSA2_REQUIRE_I32(p)                                                         \
+  do {                                                                             \
+    if ((p) == nullptr) return ::csa2::fail(CSA2_ERR_INVALID_ARG, "%s is NULL", #p); \
+    if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)                                  \
+      return ::csa2::fail(CSA2_ERR_ALIGNMENT, "%s is not 4-byte aligned", #p);       \
+  } while (0)
+
+static csa2_status check_shard(const csa2_cp_shard* sh) {
+  CSA2_REQUIRE(sh != nullptr, CSA2_ERR_INVALID_ARG, "shard is NULL");
+  CSA2_REQUIRE(sh->world >= 1 && sh->world <= CSA2_CP_MAX_WORLD, CSA2_ERR_SHAPE,
+               "world = %d outside [1, %d]", sh->world, (int)CSA2_CP_MAX_WORLD);
+  CSA2_REQUIRE(sh->rank >= 0 && sh->rank < sh->world, CSA2_ERR_INVALID_ARG,
+               "rank = %d outside [0, %d)", sh->rank, sh->world);
+  CSA2_REQUIRE(sh->shard_rows > 0 && sh->shard_rows % 128 == 0, CSA2_ERR_SHAPE,
+               "shard_rows = %d is not a positive multiple of 128", sh->shard_rows);
+  CSA2_REQUIRE((int64_t)sh->world * sh->shard_rows <= CSA2_MAX_ROWS, CSA2_ERR_SHAPE,
+               "world x shard_rows = %lld > %d", (long long)sh->world * sh->shard_rows,
+               (int)CSA2_MAX_ROWS);
+  return CSA2_OK;
+}
+
+static csa2_status check_shard_kv(const csa2_cp_shard* sh, const csa2_kv_view* kv) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  if ((r = check_kv(kv))) return r;
+  CSA2_REQUIRE(kv->max_rows <= sh->shard_rows, CSA2_ERR_SHAPE,
+               "kv->max_rows = %d > shard_rows = %d", kv->max_rows, sh->shard_rows);
+  return CSA2_OK;
+}
+
+static int cp_nsplit(int batch, int n_layers) {
+  const int ns = attn_nsplit(batch * n_layers, num_sms());
+  return ns < 2 ? 2 : ns;  // the partials must stay unmerged for the exchange
+}
+
+struct CpWs {
+  uint32_t* status;
+  int32_t* sel;        // [batch][top_k] local Top-k
+  int32_t* sel_count;  // [batch]
+  float* part_o;       // attention split partials
+  float* part_ml;
+  float* bm;           // [batch][world * S / 8] regrouped block maxima
+  int nsplit;
+  size_t bytes;
+};
+
+static CpWs cp_ws_layout(const csa2_cp_shard* sh, int batch, int n_layers, int top_k,
+                         uint8_t* base) {
+  CpWs w{};
+  w.nsplit = cp_nsplit(batch, n_layers);
+  size_t off = CSA2_WS_HEADER;
+  w.status = reinterpret_cast<uint32_t*>(base);
+  w.sel = reinterpret_cast<int32_t*>(base + off);
+  off = align256(off + (size_t)batch * top_k * sizeof(int32_t));
+  w.sel_count = reinterpret_cast<int32_t*>(base + off);
+  off = align256(off + (size_t)batch * sizeof(int32_t));
+  const size_t slots = (size_t)batch * n_layers * w.nsplit;
+  w.part_o = reinterpret_cast<float*>(base + off);
+  w.part_ml = reinterpret_cast<float*>(base + off + slots * CSA2_H * CSA2_D * sizeof(float));
+  off = align256(off + attn_partial_bytes(batch, n_layers, w.nsplit));
+  w.bm = reinterpret_cast<float*>(base + off);
+  off = align256(off + (size_t)batch * sh->world * (sh->shard_rows / CSA2_BLK) * sizeof(float));
+  w.bytes = off;
+  return w;
+}
 
 }  // namespace csa2
 
@@ -521,5 +587,295 @@ csa2_status csa2_cache_append(const csa2_kv_view* kv, const uint16_t* x, const u
   return CSA2_OK;
 }
 
+// ------------------------------------------------- context-parallel decode
+size_t csa2_cp_workspace_size(const csa2_cp_shard* sh, int32_t batch, int32_t n_layers,
+                              int32_t top_k) {
+  if (check_shard(sh) != CSA2_OK || batch < 1 || n_layers < 1 || top_k < 1) return 0;
+  return cp_ws_layout(sh, batch, n_layers, top_k, nullptr).bytes;
+}
+
+size_t csa2_cp_partial_floats(int32_t batch, int32_t n_layers) {
+  if (batch < 1 || n_layers < 1) return 0;
+  return (size_t)n_layers * batch * CSA2_H * (CSA2_D + 2);
+}
+
+csa2_status csa2_cp_local_rows(const csa2_cp_shard* sh, const int32_t* n_rows, int32_t batch,
+                               int32_t* local_rows, void* ws, size_t ws_bytes,
+                               csa2_stream_t stream) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  CSA2_REQUIRE_I32(n_rows);
+  CSA2_REQUIRE_I32(local_rows);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
+  CSA2_CUDA(launch_cp_local_rows(n_rows, batch, (int64_t)sh->rank * sh->shard_rows,
+                                 sh->shard_rows, local_rows, static_cast<uint32_t*>(ws),
+                                 (cudaStream_t)stream));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_block_max(const csa2_cp_shard* sh, const csa2_kv_view* kv,
+                              const uint16_t* q_idx, const float* w, float* bm, void* ws,
+                              size_t ws_bytes, csa2_stream_t stream) {
+  csa2_status r = check_shard_kv(sh, kv);
+  if (r) return r;
+  CSA2_REQUIRE_PTR(q_idx);
+  CSA2_REQUIRE_PTR(w);
+  CSA2_REQUIRE_PTR(bm);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  cudaStream_t st = (cudaStream_t)stream;
+  IndexWs iw{};
+  iw.status = static_cast<uint32_t*>(ws);
+  iw.bm = bm;
+  iw.bm_stride = sh->shard_rows / CSA2_BLK;
+  CUtensorMap map_k, map_q;
+  if ((r = map_rows64(&map_k, kv->idx_k, (uint64_t)kv->pool_rows, 64))) return r;
+  if ((r = map_rows64(&map_q, q_idx, (uint64_t)kv->batch * CSA2_HI, scan_query_rows(1)))) return r;
+  ScanParams sp = scan_params(kv, w, iw, 1);
+  trace_mark("scan", st);
+  CSA2_CUDA(launch_scan(map_k, map_q, sp, num_sms(), st));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_pool(const csa2_cp_shard* sh, const float* bm_all, const int32_t* n_rows,
+                         int32_t batch, int32_t P, int32_t* pool, int32_t* pool_count, void* ws,
+                         size_t ws_bytes, csa2_stream_t stream) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  CSA2_REQUIRE_PTR(bm_all);
+  CSA2_REQUIRE_I32(n_rows);
+  CSA2_REQUIRE_I32(pool);
+  CSA2_REQUIRE_I32(pool_count);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
+  CSA2_REQUIRE(P >= 1 && P <= CSA2_MAX_POOL, CSA2_ERR_SHAPE, "P = %d outside [1, %d]", P,
+               (int)CSA2_MAX_POOL);
+  const CpWs lay = cp_ws_layout(sh, batch, 1, 1, static_cast<uint8_t*>(ws));
+  const int nb = sh->shard_rows / CSA2_BLK;
+  const bool regroup = sh->world > 1 && batch > 1;
+  CSA2_REQUIRE(ws_bytes >= (regroup ? lay.bytes : (size_t)CSA2_WS_HEADER), CSA2_ERR_WORKSPACE,
+               "workspace %zu < %zu bytes", ws_bytes, regroup ? lay.bytes : (size_t)CSA2_WS_HEADER);
+  cudaStream_t st = (cudaStream_t)stream;
+  const float* bm = bm_all;
+  if (regroup) {
+    CSA2_CUDA(launch_cp_bm_regroup(bm_all, sh->world, batch, nb, lay.bm, st));
+    bm = lay.bm;
+  }
+  trace_mark("block_select", st);
+  CSA2_CUDA(launch_block_select(bm, sh->world * nb, n_rows, sh->world * sh->shard_rows, batch, 1,
+                                P, pool, P, pool_count, lay.status, st));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_filter(const csa2_cp_shard* sh, int32_t unit, const int32_t* list,
+                           const int32_t* count, int32_t stride, int32_t batch, int32_t* out,
+                           int32_t* out_count, int32_t out_stride, int32_t* copy,
+                           int32_t* copy_count, void* ws, size_t ws_bytes,
+                           csa2_stream_t stream) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  CSA2_REQUIRE(unit == 1 || unit == CSA2_BLK, CSA2_ERR_INVALID_ARG, "unit = %d (1 or %d)", unit,
+               (int)CSA2_BLK);
+  CSA2_REQUIRE_I32(list);
+  CSA2_REQUIRE_I32(count);
+  CSA2_REQUIRE_I32(out);
+  CSA2_REQUIRE_I32(out_count);
+  CSA2_REQUIRE((copy == nullptr) == (copy_count == nullptr), CSA2_ERR_INVALID_ARG,
+               "copy and copy_count must both be given or both be NULL");
+  if (copy) {
+    CSA2_REQUIRE_I32(copy);
+    CSA2_REQUIRE_I32(copy_count);
+  }
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
+  CSA2_REQUIRE(stride >= 1 && stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
+               "stride = %d outside [1, %d]", stride, (int)CSA2_MAX_POOL);
+  CSA2_REQUIRE(out_stride >= 1 && out_stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
+               "out_stride = %d outside [1, %d]", out_stride, (int)CSA2_MAX_POOL);
+  CpFilterParams p{};
+  p.list = list;
+  p.count = count;
+  p.stride = stride;
+  p.lo = sh->rank * (sh->shard_rows / unit);
+  p.hi = p.lo + sh->shard_rows / unit;
+  p.out = out;
+  p.out_count = out_count;
+  p.out_stride = out_stride;
+  p.copy = copy;
+  p.copy_count = copy_count;
+  p.status = static_cast<uint32_t*>(ws);
+  CSA2_CUDA(launch_cp_filter(p, batch, (cudaStream_t)stream));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_select_local(const csa2_cp_shard* sh, const csa2_kv_view* kv,
+                                 const uint16_t* q_idx, const float* w, const int32_t* cand,
+                                 const int32_t* cand_count, int32_t cand_stride, int32_t top_k,
+                                 uint32_t* send, void* ws, size_t ws_bytes,
+                                 csa2_stream_t stream) {
+  csa2_status r = check_shard_kv(sh, kv);
+  if (r) return r;
+  if ((r = check_topk(top_k, 0))) return r;
+  CSA2_REQUIRE_PTR(q_idx);
+  CSA2_REQUIRE_PTR(w);
+  CSA2_REQUIRE_I32(cand);
+  CSA2_REQUIRE_I32(cand_count);
+  CSA2_REQUIRE(send != nullptr && (reinterpret_cast<uintptr_t>(send) & 7u) == 0,
+               CSA2_ERR_ALIGNMENT, "send is NULL or not 8-byte aligned");
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(cand_stride >= 1 && cand_stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
+               "cand_stride = %d outside [1, %d]", cand_stride, (int)CSA2_MAX_POOL);
+  const CpWs lay = cp_ws_layout(sh, kv->batch, 1, top_k, static_cast<uint8_t*>(ws));
+  const size_t need = reinterpret_cast<uint8_t*>(lay.part_o) - static_cast<uint8_t*>(ws);
+  CSA2_REQUIRE(ws_bytes >= need, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  RescoreParams rp = rescore_params(kv, cand, cand_count, cand_stride, top_k, lay.status);
+  rp.job[0] = RescoreJob{q_idx, w, lay.sel, lay.sel_count, top_k};
+  trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, 1, kv->batch, cand_blocks_max(kv, cand_stride), st));
+  CpExportParams xp{};
+  xp.idx_k = kv->idx_k;
+  xp.page_table = kv->page_table;
+  xp.max_pages = kv->max_pages;
+  xp.max_rows = kv->max_rows;
+  xp.seq_stride = kv->seq_stride;
+  xp.pool_rows = kv->pool_rows;
+  xp.n_rows = kv->n_rows;
+  xp.q_idx = q_idx;
+  xp.w = w;
+  xp.idx = lay.sel;
+  xp.idx_count = lay.sel_count;
+  xp.top_k = top_k;
+  xp.pos_base = sh->rank * sh->shard_rows;
+  xp.send = reinterpret_cast<uint2*>(send);
+  xp.status = lay.status;
+  CSA2_CUDA(launch_cp_export(xp, kv->batch, st));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_select_merge(const csa2_cp_shard* sh, const uint32_t* gathered,
+                                 int32_t n_jobs, int32_t job, int32_t batch, int32_t top_k,
+                                 int32_t* idx, int32_t* idx_count, void* ws, size_t ws_bytes,
+                                 csa2_stream_t stream) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  if ((r = check_topk(top_k, 0))) return r;
+  CSA2_REQUIRE(gathered != nullptr && (reinterpret_cast<uintptr_t>(gathered) & 7u) == 0,
+               CSA2_ERR_ALIGNMENT, "gathered is NULL or not 8-byte aligned");
+  CSA2_REQUIRE_I32(idx);
+  CSA2_REQUIRE_I32(idx_count);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
+  CSA2_REQUIRE(n_jobs >= 1 && job >= 0 && job < n_jobs, CSA2_ERR_INVALID_ARG,
+               "job = %d, n_jobs = %d", job, n_jobs);
+  CSA2_REQUIRE(sh->world * top_k <= cp_merge_capacity(), CSA2_ERR_SHAPE,
+               "world x top_k = %d > %d", sh->world * top_k, cp_merge_capacity());
+  CpMergeParams p{};
+  p.gathered = reinterpret_cast<const uint2*>(gathered);
+  p.world = sh->world;
+  p.n_jobs = n_jobs;
+  p.job = job;
+  p.batch = batch;
+  p.top_k = top_k;
+  p.idx = idx;
+  p.idx_count = idx_count;
+  CSA2_CUDA(launch_cp_merge_select(p, (cudaStream_t)stream));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_attn_partial(const csa2_cp_shard* sh, const csa2_kv_view* kv,
+                                 int32_t n_layers, const uint16_t* q, const uint8_t* swa,
+                                 const int32_t* swa_len, const int32_t* idx_local,
+                                 const int32_t* idx_count, int32_t idx_stride, float sm_scale,
+                                 float* partial, void* ws, size_t ws_bytes,
+                                 csa2_stream_t stream) {
+  csa2_status r = check_shard_kv(sh, kv);
+  if (r) return r;
+  CSA2_REQUIRE(n_layers >= 1 && n_layers <= AT_MAX_LAYERS, CSA2_ERR_SHAPE,
+               "n_layers = %d outside [1, %d]", n_layers, AT_MAX_LAYERS);
+  CSA2_REQUIRE_PTR(q);
+  CSA2_REQUIRE_PTR(swa);
+  CSA2_REQUIRE_I32(swa_len);
+  CSA2_REQUIRE_I32(idx_local);
+  CSA2_REQUIRE_I32(idx_count);
+  CSA2_REQUIRE_PTR(partial);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(idx_stride >= 1 && idx_stride <= CSA2_MAX_TOPK, CSA2_ERR_SHAPE,
+               "idx_stride = %d outside [1, %d]", idx_stride, (int)CSA2_MAX_TOPK);
+  CSA2_REQUIRE(sm_scale == sm_scale, CSA2_ERR_INVALID_ARG, "sm_scale is NaN");
+  const int B = kv->batch;
+  const CpWs lay = cp_ws_layout(sh, B, n_layers, 1, static_cast<uint8_t*>(ws));
+  const size_t need = reinterpret_cast<uint8_t*>(lay.bm) - static_cast<uint8_t*>(ws);
+  CSA2_REQUIRE(ws_bytes >= need, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  AttnParams ap{};
+  fill_attn_common(ap, kv, swa_len, sm_scale, idx_stride);
+  ap.n_layers = n_layers;
+  ap.nsplit = lay.nsplit;
+  ap.part_o = lay.part_o;
+  ap.part_ml = lay.part_ml;
+  ap.status = lay.status;
+  for (int l = 0; l < n_layers; l++)
+    ap.layer[l] = AttnLayer{q + (size_t)l * B * CSA2_H * CSA2_D,
+                            swa + (size_t)l * B * CSA2_W * CSA2_D,
+                            idx_local + (size_t)l * B * idx_stride,
+                            idx_count + (size_t)l * B,
+                            nullptr,
+                            nullptr,
+                            nullptr};  // nsplit >= 2: the output is never written here
+  CSA2_CUDA(launch_attn(ap, st, /*merge=*/false));
+  const size_t o_floats = (size_t)n_layers * B * CSA2_H * CSA2_D;
+  CpAttnMergeParams mp{};
+  mp.part_o = lay.part_o;
+  mp.part_ml = lay.part_ml;
+  mp.o_pstride = CSA2_H * CSA2_D;
+  mp.o_sstride = (int64_t)lay.nsplit * CSA2_H * CSA2_D;
+  mp.ml_pstride = CSA2_H * 2;
+  mp.ml_sstride = (int64_t)lay.nsplit * CSA2_H * 2;
+  mp.nparts = lay.nsplit;
+  mp.batch = B;
+  mp.out_o = partial;
+  mp.out_ml = partial + o_floats;
+  CSA2_CUDA(launch_cp_attn_merge(mp, n_layers, false, st));
+  return CSA2_OK;
+}
+
+csa2_status csa2_cp_attn_combine(const csa2_cp_shard* sh, const float* gathered,
+                                 int32_t n_layers, int32_t batch, uint16_t* out, void* ws,
+                                 size_t ws_bytes, csa2_stream_t stream) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  CSA2_REQUIRE_PTR(gathered);
+  CSA2_REQUIRE_PTR(out);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
+  CSA2_REQUIRE(n_layers >= 1 && n_layers <= 65535, CSA2_ERR_SHAPE, "n_layers = %d", n_layers);
+  CSA2_REQUIRE(sh->world <= CP_MAX_PARTS, CSA2_ERR_SHAPE, "world = %d > %d", sh->world,
+               CP_MAX_PARTS);
+  const size_t per_rank = csa2_cp_partial_floats(batch, n_layers);
+  const size_t o_floats = (size_t)n_layers * batch * CSA2_H * CSA2_D;
+  CpAttnMergeParams mp{};
+  mp.part_o = gathered;
+  mp.part_ml = gathered + o_floats;
+  mp.o_pstride = (int64_t)per_rank;
+  mp.o_sstride = CSA2_H * CSA2_D;
+  mp.ml_pstride = (int64_t)per_rank;
+  mp.ml_sstride = CSA2_H * 2;
+  mp.nparts = sh->world;
+  mp.batch = batch;
+  mp.out = out;
+  CSA2_CUDA(launch_cp_attn_merge(mp, n_layers, true, (cudaStream_t)stream));
+  return CSA2_OK;
+}
 
 }  // extern "C"

@@ -129,7 +129,8 @@ struct AttnParams {
 };
 int attn_nsplit(int pairs, int num_sms);
 size_t attn_partial_bytes(int batch, int n_layers, int nsplit);
-cudaError_t launch_attn(const AttnParams& p, cudaStream_t st);
+// merge = false leaves the split partials in part_o / part_ml (nsplit > 1).
+cudaError_t launch_attn(const AttnParams& p, cudaStream_t st, bool merge = true);
 
 // ------------------------------------------------------------ cache append
 struct AppendParams {
@@ -152,5 +153,62 @@ struct AppendParams {
   uint32_t* status;
 };
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
+
+// ------------------------------------------------- context-parallel decode
+constexpr int CP_MAX_PARTS = 16;  // shards (and attention splits) one merge combines
+struct CpFilterParams {
+  const int32_t* list;   // [batch][stride] ascending ids
+  const int32_t* count;  // [batch]
+  int32_t stride;        // <= CSA2_MAX_POOL
+  int32_t lo, hi;        // kept: lo <= id < hi, written as id - lo
+  int32_t* out;          // [batch][out_stride]
+  int32_t* out_count;    // [batch]
+  int32_t out_stride;
+  int32_t* copy;         // optional verbatim copy of list / count
+  int32_t* copy_count;
+  uint32_t* status;
+};
+struct CpExportParams {
+  const uint16_t* idx_k;
+  const int32_t* page_table;
+  int32_t max_pages;
+  int32_t max_rows;
+  int64_t seq_stride;
+  int64_t pool_rows;
+  const int32_t* n_rows;     // this shard's visible rows per sequence
+  const uint16_t* q_idx;     // [batch][8][64]
+  const float* w;            // [batch][8]
+  const int32_t* idx;        // [batch][top_k] local positions, ascending
+  const int32_t* idx_count;  // [batch]
+  int32_t top_k;
+  int32_t pos_base;          // global position of local position 0
+  uint2* send;               // [batch][top_k] (key, global position)
+  uint32_t* status;
+};
+struct CpMergeParams {
+  const uint2* gathered;  // [world][n_jobs][batch][top_k]
+  int32_t world, n_jobs, job, batch, top_k;
+  int32_t* idx;           // [batch][top_k]
+  int32_t* idx_count;     // [batch]
+};
+struct CpAttnMergeParams {
+  const float* part_o;
+  const float* part_ml;
+  int64_t o_pstride, o_sstride, ml_pstride, ml_sstride;  // floats
+  int32_t nparts, batch;
+  float* out_o;      // merged partials [slot][16][512] (local merge)
+  float* out_ml;     // [slot][16][2]
+  uint16_t* out;     // bf16 [slot][16][512] (final merge)
+};
+cudaError_t launch_cp_local_rows(const int32_t* n_rows, int batch, int64_t lo, int shard_rows,
+                                 int32_t* local_rows, uint32_t* status, cudaStream_t st);
+cudaError_t launch_cp_bm_regroup(const float* src, int world, int batch, int nb, float* dst,
+                                 cudaStream_t st);
+cudaError_t launch_cp_filter(const CpFilterParams& p, int batch, cudaStream_t st);
+cudaError_t launch_cp_export(const CpExportParams& p, int batch, cudaStream_t st);
+cudaError_t launch_cp_merge_select(const CpMergeParams& p, cudaStream_t st);
+cudaError_t launch_cp_attn_merge(const CpAttnMergeParams& p, int n_layers, bool final_out,
+                                 cudaStream_t st);
+int cp_merge_capacity();
 
 }  // namespace csa2

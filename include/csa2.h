@@ -351,6 +351,135 @@ size_t csa2_group_workspace_size(const csa2_group_desc *desc);
 csa2_status csa2_layer_group(const csa2_group_desc *desc, void *ws, size_t ws_bytes,
                              csa2_stream_t stream);
 
+/* ------------------------------------------------ context-parallel decode */
+
+/*
+ * One decode step of a layer group with every sequence's positions cut into
+ * `world` contiguous shards of shard_rows (S) rows: rank r holds positions
+ * [r*S, (r+1)*S) of every sequence in its own cache, a csa2_kv_view whose
+ * n_rows are the shard's visible rows (csa2_cp_local_rows) and whose
+ * max_rows <= S.  Scores, block maxima and attention rows are per position,
+ * and every selection of the step is a Top-k under one total order (the key,
+ * then the lower position or block) [REL §CSA2; YOM §二 mode table and HSI
+ * paragraph], so the step is local work on each shard plus three exchanges.
+ * The caller runs each exchange as an all-gather over the ranks in rank
+ * order (NCCL over NVLink, or any transport): the library moves no data
+ * between ranks and never waits on another rank.
+ *   1. FULL layer (and REINDEX without a pool): csa2_cp_block_max ->
+ *      all-gather -> csa2_cp_pool: the pool (P = pool_blocks, or top_k
+ *      blocks without a pool), the same on every rank.
+ *   2. Selection: csa2_cp_filter (unit 8: the pool blocks this shard owns) ->
+ *      csa2_cp_select_local -> all-gather -> csa2_cp_select_merge: the
+ *      layer's Top-k positions, the same on every rank and equal to the
+ *      one-GPU csa2_layer_group result (the keys exchanged are bit-identical
+ *      to those the one-GPU rescore ranks).
+ *   3. Attention: csa2_cp_filter (unit 1: the selected rows this shard owns)
+ *      -> csa2_cp_attn_partial -> all-gather -> csa2_cp_attn_combine.
+ * The sliding window lives on one rank: pass the window lengths there and
+ * zeros on the others.  Every call is asynchronous on its stream and records
+ * device checks in the status word of ws, like the rest of this ABI.
+ * Count arrays (n_rows, counts, index lists) need 4-byte alignment only.
+ */
+enum { CSA2_CP_MAX_WORLD = 16 };
+
+typedef struct {
+  int32_t rank;       /* this shard, 0 <= rank < world                          */
+  int32_t world;      /* shards, 1 <= world <= CSA2_CP_MAX_WORLD                 */
+  int32_t shard_rows; /* S: a multiple of 128; world * S <= CSA2_MAX_ROWS        */
+} csa2_cp_shard;
+
+/* Bytes of workspace that every csa2_cp_* call of one rank needs for a group
+ * of n_layers layers (status word, local selection scratch, attention split
+ * partials, regrouped block maxima).  0 on a bad argument. */
+size_t csa2_cp_workspace_size(const csa2_cp_shard *sh, int32_t batch, int32_t n_layers,
+                              int32_t top_k);
+
+/* Floats in one rank's attention partial: n_layers * batch * 16 * (512 + 2). */
+size_t csa2_cp_partial_floats(int32_t batch, int32_t n_layers);
+
+/* local_rows[b] = clamp(n_rows[b] - rank * S, 0, S): the shard's visible rows.
+ * n_rows, local_rows: device int32 [batch].  A negative n_rows[b] is a device
+ * check. */
+csa2_status csa2_cp_local_rows(const csa2_cp_shard *sh, const int32_t *n_rows, int32_t batch,
+                               int32_t *local_rows, void *ws, size_t ws_bytes,
+                               csa2_stream_t stream);
+
+/* Block maxima over the shard: bm[b][j] = max of the score
+ * s = sum_h w_h * relu(q_idx_h . k) over the shard's visible rows 8j..8j+7
+ * [YOM §二 HSI], by the same scan as csa2_index_full.  q_idx bf16
+ * [batch][8][64], w fp32 [batch][8], bm fp32 [batch][S / 8] (entries at or
+ * past the visible blocks are left as they are).  kv: this shard's view. */
+csa2_status csa2_cp_block_max(const csa2_cp_shard *sh, const csa2_kv_view *kv,
+                              const uint16_t *q_idx, const float *w, float *bm, void *ws,
+                              size_t ws_bytes, csa2_stream_t stream);
+
+/* The pool from the all-gathered block maxima bm_all fp32 [world][batch][S/8]
+ * (rank-major, as an all-gather of every rank's bm lays them out): the top P
+ * blocks by block maximum over the blocks of the global visible rows n_rows
+ * (int32 [batch]), ties to the lower block.  pool int32 [batch][P] ascending
+ * global block ids, -1 padded; pool_count int32 [batch].  P in
+ * [1, CSA2_MAX_POOL]. */
+csa2_status csa2_cp_pool(const csa2_cp_shard *sh, const float *bm_all, const int32_t *n_rows,
+                         int32_t batch, int32_t P, int32_t *pool, int32_t *pool_count,
+                         void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* The ids in list that this shard owns, made local.  unit = 8 for block ids
+ * (shard range [rank*S/8, (rank+1)*S/8)), 1 for positions ([rank*S,
+ * (rank+1)*S)).  out[b] = the ids x of list[b][0 .. count[b]) in the range,
+ * as x - range start, in list order, -1 padded to out_stride; out_count[b]
+ * their number (at most out_stride).  copy and copy_count (both or neither)
+ * receive list [batch][stride] and count verbatim.  stride and out_stride in
+ * [1, CSA2_MAX_POOL]; a count outside [0, stride] is a device check. */
+csa2_status csa2_cp_filter(const csa2_cp_shard *sh, int32_t unit, const int32_t *list,
+                           const int32_t *count, int32_t stride, int32_t batch, int32_t *out,
+                           int32_t *out_count, int32_t out_stride, int32_t *copy,
+                           int32_t *copy_count, void *ws, size_t ws_bytes,
+                           csa2_stream_t stream);
+
+/* The shard's Top-k among its candidate blocks cand int32 [batch][cand_stride]
+ * (local block ids, ascending; cand_count [batch]), scored with q_idx / w as
+ * in csa2_index_reindex, exported for the merge: send uint32
+ * [batch][top_k][2] = (key, global position) in ascending position, then
+ * (0, 0xFFFFFFFF).  The key is the fp32 score mapped to an unsigned integer
+ * of the same order (0 is never a key).  send: 8-byte aligned. */
+csa2_status csa2_cp_select_local(const csa2_cp_shard *sh, const csa2_kv_view *kv,
+                                 const uint16_t *q_idx, const float *w, const int32_t *cand,
+                                 const int32_t *cand_count, int32_t cand_stride, int32_t top_k,
+                                 uint32_t *send, void *ws, size_t ws_bytes,
+                                 csa2_stream_t stream);
+
+/* The global Top-k of job `job` (ties to the lower position) from the
+ * all-gathered exports gathered uint32 [world][n_jobs][batch][top_k][2]
+ * (several layers' exports may share one all-gather).  idx int32
+ * [batch][top_k] ascending global positions, -1 padded; idx_count [batch].
+ * world * top_k <= 8192. */
+csa2_status csa2_cp_select_merge(const csa2_cp_shard *sh, const uint32_t *gathered,
+                                 int32_t n_jobs, int32_t job, int32_t batch, int32_t top_k,
+                                 int32_t *idx, int32_t *idx_count, void *ws, size_t ws_bytes,
+                                 csa2_stream_t stream);
+
+/* The shard's attention partial for every layer: over its selected rows
+ * idx_local int32 [L][batch][idx_stride] (local positions from csa2_cp_filter,
+ * counts idx_count [L][batch]) and the window rows swa_len[b] (zeros on ranks
+ * without the window), the unnormalised softmax numerator and its (max, sum)
+ * per head, as csa2_sparse_attn_decode computes them before normalising.
+ * q bf16 [L][batch][16][512], swa E4M3 [L][batch][128][512].  partial fp32
+ * [csa2_cp_partial_floats]: O [L][batch][16][512], then (max in log2 units of
+ * sm_scale * q.k, sum) [L][batch][16][2].  n_layers <= 32. */
+csa2_status csa2_cp_attn_partial(const csa2_cp_shard *sh, const csa2_kv_view *kv,
+                                 int32_t n_layers, const uint16_t *q, const uint8_t *swa,
+                                 const int32_t *swa_len, const int32_t *idx_local,
+                                 const int32_t *idx_count, int32_t idx_stride, float sm_scale,
+                                 float *partial, void *ws, size_t ws_bytes,
+                                 csa2_stream_t stream);
+
+/* out bf16 [L][batch][16][512] from the all-gathered partials gathered fp32
+ * [world][csa2_cp_partial_floats]: the log-sum-exp merge over the ranks,
+ * zeros where no rank had a key. */
+csa2_status csa2_cp_attn_combine(const csa2_cp_shard *sh, const float *gathered,
+                                 int32_t n_layers, int32_t batch, uint16_t *out, void *ws,
+                                 size_t ws_bytes, csa2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

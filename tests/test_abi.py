@@ -62,3 +62,35 @@ def test_group_host_validation(lib):
     desc.n_layers = 1
     assert lib2.csa2_layer_group(ctypes.byref(desc), None, 0, None) != 0
     assert lib2.csa2_group_workspace_size(ctypes.byref(desc)) == 0
+
+
+def test_cp_host_validation(lib):
+    """Shard and argument checks of the context-parallel entry points run on
+    the host, before any CUDA call."""
+    from fp4_kv_cache_quantize_b200 import csa2
+    lib2 = csa2._lib
+    bad = [csa2.CpShard(0, 2, 100), csa2.CpShard(2, 2, 128), csa2.CpShard(-1, 2, 128),
+           csa2.CpShard(0, 17, 128), csa2.CpShard(0, 2, 1 << 20), csa2.CpShard(0, 0, 128)]
+    for sh in bad:
+        assert csa2.csa2_cp_workspace_size(sh, 1, 1, 512) == 0
+        assert lib2.csa2_cp_local_rows(ctypes.byref(sh), None, 1, None, None, 0, None) != 0
+    assert lib2.csa2_cp_local_rows(None, None, 1, None, None, 0, None) == 1
+    assert csa2.csa2_cp_partial_floats(2, 20) == 20 * 2 * 16 * 514
+    assert csa2.csa2_cp_partial_floats(0, 20) == 0
+    sh = csa2.CpShard(0, 2, 128)
+    p = ctypes.c_void_p(256)
+    f = lib2.csa2_cp_filter
+    # unit other than 1 or 8
+    assert f(ctypes.byref(sh), 3, p, p, 1, 1, p, p, 1, None, None, p, 256, None) == 1
+    # copy without copy_count
+    assert f(ctypes.byref(sh), 1, p, p, 1, 1, p, p, 1, p, None, p, 256, None) == 1
+    # stride beyond the pool bound
+    assert f(ctypes.byref(sh), 1, p, p, 4096, 1, p, p, 1, None, None, p, 256, None) == 2
+    # misaligned count array
+    assert f(ctypes.byref(sh), 1, p, ctypes.c_void_p(258), 1, 1, p, p, 1, None, None, p, 256,
+             None) == 3
+    m = lib2.csa2_cp_select_merge
+    assert m(ctypes.byref(sh), p, 1, 1, 1, 512, p, p, p, 256, None) == 1   # job >= n_jobs
+    assert m(ctypes.byref(sh), ctypes.c_void_p(260), 1, 0, 1, 512, p, p, p, 256, None) == 3
+    assert m(ctypes.byref(sh), p, 1, 0, 1, 513, p, p, p, 256, None) == 2   # top_k > 512
+

@@ -1,0 +1,146 @@
+"""GPU parity of the context-parallel decode step (csa2_cp_* entry points,
+driven by fp4_kv_cache_quantize_b200.cp) with every shard run on one device
+through LocalComm.  For 1 to 4 shards, contiguous and paged caches, with and
+without the HSI pool:
+  * every shard's indices and pool equal the one-device csa2_layer_group's
+    exactly (the shards exchange keys bit-identical to the ones the
+    one-device rescore ranks, and the merge keeps its tie rule);
+  * indices, pool and attention output match the oracle's layer group under
+    the usual tolerances (ties within 1e-5; attention relative L2 <= 5e-3).
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp4_kv_cache_quantize_b200 import synth
+from gpu_helpers import ATTN_RTOL, DeviceWorkload, bf16_to_f64, rel_l2
+from test_gpu_group import compare_group
+
+pytestmark = pytest.mark.gpu
+FULL, REINDEX, REUSE = 0, 1, 2
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fp4_kv_cache_quantize_b200 import csa2
+    return csa2
+
+
+def relayout(dw, stride):
+    """The workload's cache with sequence b at rows [b * stride, ...)."""
+    wl = dw.wl
+    rows = wl.B * stride
+    codes = torch.zeros((rows, 256), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((rows, 32), dtype=torch.uint8, device="cuda")
+    idxk = torch.zeros((rows, 64), dtype=torch.int16, device="cuda")
+    for b in range(wl.B):
+        n = int(wl.n_rows[b])
+        src = torch.from_numpy(wl.row_of(b, np.arange(n))).cuda()
+        codes[b * stride:b * stride + n] = dw.codes[src]
+        scales[b * stride:b * stride + n] = dw.scales[src]
+        idxk[b * stride:b * stride + n] = dw.idxk[src]
+    return codes, scales, idxk
+
+
+def run_cp(lib, dw, world, *, paged):
+    from fp4_kv_cache_quantize_b200 import cp
+    wl = dw.wl
+    S = cp.shard_rows_for(int(wl.n_rows.max()), world)
+    if paged:
+        codes, scales, idxk, stride, pt = dw.codes, dw.scales, dw.idxk, 0, dw.page_table
+    else:
+        stride = world * S
+        codes, scales, idxk = relayout(dw, stride)
+        pt = None
+    ranks = []
+    for r in range(world):
+        kv = cp.local_view(codes, scales, idxk, rank=r, world=world, shard_rows=S, batch=wl.B,
+                           seq_stride=stride, page_table=pt)
+        ranks.append(cp.CPRank(kv, rank=r, world=world, shard_rows=S, n_layers=wl.L,
+                               top_k=wl.top_k, pool_blocks=wl.pool_blocks))
+    cp.cp_layer_group(ranks, cp.LocalComm(world), wl.modes, dw.n_rows, dw.q_idx, dw.w, dw.q,
+                      dw.swa, dw.swa_len, sm_scale=float(np.float32(512 ** -0.5)))
+    for r in ranks:
+        lib.csa2_sync_status(r.ws)
+    return ranks
+
+
+def one_device(lib, dw):
+    wl = dw.wl
+    grp = lib.LayerGroup(dw.kv, wl.modes, dw.q_idx, dw.w, dw.q, dw.swa, dw.swa_len,
+                         top_k=wl.top_k, pool_blocks=wl.pool_blocks,
+                         sm_scale=float(np.float32(512 ** -0.5)))
+    ws = lib.workspace(grp.workspace_size())
+    lib.csa2_layer_group(grp, ws)
+    lib.csa2_sync_status(ws)
+    return grp
+
+
+def check(lib, orc, wl, world, paged):
+    dw = DeviceWorkload(lib, wl, orc)
+    ranks = run_cp(lib, dw, world, paged=paged)
+    grp = one_device(lib, dw)
+    for r in ranks:
+        assert torch.equal(r.idx_count, grp.idx_count), r.shard.rank
+        for l in range(wl.L):
+            for b in range(wl.B):
+                n = int(grp.idx_count[l, b])
+                assert torch.equal(r.idx[l, b], grp.idx[l, b]), (r.shard.rank, l, b, n)
+        if wl.pool_blocks:
+            assert torch.equal(r.pool_count, grp.pool_count)
+            assert torch.equal(r.pool, grp.pool)
+        # the shards' outputs agree with the one-device step to bf16 rounding
+        err = rel_l2(bf16_to_f64(r.out), bf16_to_f64(grp.out))
+        assert err <= ATTN_RTOL, (r.shard.rank, err)
+    compare_group(orc, dw, ranks[0])
+    compare_group(orc, dw, ranks[-1])
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+def test_cp_contiguous_hsi_group(lib, orc, world):
+    wl = synth.make("cp", seed=500 + world, B=2, n_rows=[20000, 300],
+                    modes=[FULL, REUSE, REINDEX, REUSE, FULL, REINDEX], pool_blocks=2048,
+                    swa_len=[128, 37])
+    check(lib, orc, wl, world, paged=False)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_cp_paged_without_pool(lib, orc, world):
+    wl = synth.make("cp", seed=520 + world, B=3, n_rows=[9000, 4099, 64],
+                    modes=[FULL, REINDEX, REUSE], pool_blocks=0, paged=True,
+                    swa_len=[128, 0, 5])
+    check(lib, orc, wl, world, paged=True)
+
+
+def test_cp_attention_only_window(lib, orc):
+    """A sequence with no global entries: every shard's rows are empty and
+    the output is the window-only attention of the rank holding the window."""
+    wl = synth.make("cp", seed=530, B=2, n_rows=[0, 700], modes=[FULL, REUSE],
+                    pool_blocks=0, swa_len=[90, 128])
+    dw = DeviceWorkload(lib, wl, orc)
+    ranks = run_cp(lib, dw, 2, paged=False)
+    kv = dw.oracle_kv(orc)
+    ref = orc.layer_group(kv, orc.dims(), wl.n_rows, wl.modes, wl.q_idx, wl.w_h, wl.q, wl.swa,
+                          wl.swa_len, top_k=wl.top_k, pool_blocks=0,
+                          sm_scale=float(np.float32(512 ** -0.5)))
+    out = bf16_to_f64(ranks[1].out)
+    for l in range(wl.L):
+        for b in range(wl.B):
+            assert rel_l2(out[l, b], ref["out"][l, b]) <= ATTN_RTOL, (l, b)
+    assert int(ranks[0].idx_count[0, 0]) == 0
+
+
+def test_cp_rejects_bad_shards(lib):
+    from fp4_kv_cache_quantize_b200 import cp
+    assert lib.csa2_cp_workspace_size(lib.CpShard(0, 2, 100), 1, 1, 512) == 0  # not x128
+    assert lib.csa2_cp_workspace_size(lib.CpShard(2, 2, 128), 1, 1, 512) == 0  # rank >= world
+    assert lib.csa2_cp_workspace_size(lib.CpShard(0, 17, 128), 1, 1, 512) == 0  # world > 16
+    assert lib.csa2_cp_workspace_size(lib.CpShard(0, 2, 1 << 20), 1, 1, 512) == 0  # > 1M rows
+    assert cp.shard_rows_for(20000, 3) == 6784
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(lib.Csa2Error) as e:
+        lib.csa2_cp_filter(lib.CpShard(0, 2, 128), 3, n.view(1, 1), n, n.view(1, 1), n,
+                           lib.workspace(256))
+    assert e.value.status == 1
