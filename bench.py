@@ -378,6 +378,58 @@ def time_multi_query(csa2, wl, kv, dev, stream, flush_l2, K, W, with_cpu, Q=4):
     return out
 
 
+def time_context_parallel(csa2, wl, bufs, grp, stream, flush_l2, K, W, world=8):
+    """The context-parallel decode step with every sequence cut into `world`
+    shards, all run on this one GPU (LocalComm: the shards' kernels back to
+    back, each exchange one device copy): its time per step, and whether its
+    indices, pool and output equal the one-device step's on the same inputs."""
+    import torch
+    from fp4_kv_cache_quantize_b200 import cp
+    codes, scales, idxk, n_rows, pt, q_idx, w_h, q, swa, swa_len = bufs
+    S = cp.shard_rows_for(int(wl.n_rows.max()), world)
+    if pt is None and wl.B > 1 and wl.seq_stride < world * S:
+        return {"skipped": "contiguous layout narrower than world x shard_rows"}
+    ranks = [cp.CPRank(cp.local_view(codes, scales, idxk, rank=r, world=world, shard_rows=S,
+                                     batch=wl.B, seq_stride=max(wl.seq_stride, world * S),
+                                     page_table=pt),
+                       rank=r, world=world, shard_rows=S, n_layers=wl.L, top_k=wl.top_k,
+                       pool_blocks=wl.pool_blocks) for r in range(world)]
+    comm = cp.LocalComm(world)
+    sm = csa2.D ** -0.5
+
+    def step():
+        cp.cp_layer_group(ranks, comm, wl.modes, n_rows, q_idx, w_h, q, swa, swa_len,
+                          sm_scale=sm)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    for r in ranks:
+        csa2.csa2_sync_status(r.ws)
+    same = all(torch.equal(r.idx, grp.idx) and torch.equal(r.idx_count, grp.idx_count)
+               for r in ranks)
+    if wl.pool_blocks:
+        same = same and all(torch.equal(r.pool, grp.pool) for r in ranks)
+    a, b = ranks[0].out.double(), grp.out.double()
+    err = float((a - b).norm() / max(float(b.norm()), 1e-30))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for i in range(K):
+        flush_l2()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(x.elapsed_time(y) for x, y in ev) / K
+    return {"world": world, "shard_rows": S, "ms_per_step_one_gpu_emulation": ms,
+            "steps": K, "warmup": W,
+            "indices_and_pool_equal_one_device": bool(same),
+            "out_rel_l2_vs_one_device": err,
+            "note": (f"{world} shards of every sequence run back to back on one GPU, each "
+                     "exchange a device copy; the time is the sum over shards plus the "
+                     "replicated merges, not a multi-GPU step time")}
+
+
 def run_gpu(args, wl, rank, world):
     import torch
 
@@ -584,6 +636,13 @@ def run_gpu(args, wl, rank, world):
     prefill = time_multi_query(csa2, wl, kv, dev, stream, flush_l2, 5, 3, with_cpu, Q=64)
     prefill["note"] = ("chunked prefill of 64 new tokens; the scan runs 8 passes of 8 queries "
                        "(MMA N = 64)")
+    try:
+        cpar = time_context_parallel(
+            csa2, wl, (codes, scales, idxk, n_rows, pt, q_idx, w_h, q, swa, swa_len), grp, stream,
+            flush_l2, 10, 3)
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        torch.cuda.synchronize()
+        cpar = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     units = wl.B * wl.L
     value = job_throughput(units, world, t_step)
@@ -621,7 +680,7 @@ def run_gpu(args, wl, rank, world):
                                "the neighbouring steps' compute; no L2 flush (134 MB of "
                                "indexer K per step exceeds the 126 MB L2)")},
             "next_rows": {"cache_append": append, "multi_query": multi,
-                          "prefill_chunk": prefill},
+                          "prefill_chunk": prefill, "context_parallel": cpar},
             "gpu_launches": int(launches * K),
             "gpu_launches_per_step": int(launches),
             "clocks": sampler.summary(),
