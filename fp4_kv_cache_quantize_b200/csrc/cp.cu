@@ -324,7 +324,7 @@ cudaError_t launch_cp_bm_regroup(const float* src, int world, int batch, int nb,
                                  cudaStream_t st) {
   const int64_t total = (int64_t)world * batch * nb;
   int64_t blocks = (total + 255) / 256;
-  if (blocks > 4 * 148) blocks = 4 * 148;
+  if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
   if (blocks < 1) blocks = 1;
   trace_mark("cp_bm_regroup", st);
   cp_bm_regroup_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, world, batch, nb, dst);
