@@ -412,22 +412,63 @@ def time_context_parallel(csa2, wl, bufs, grp, stream, flush_l2, K, W, world=8):
         same = same and all(torch.equal(r.pool, grp.pool) for r in ranks)
     a, b = ranks[0].out.double(), grp.out.double()
     err = float((a - b).norm() / max(float(b.norm()), 1e-30))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
-    for i in range(K):
-        flush_l2()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    ms = sum(x.elapsed_time(y) for x, y in ev) / K
-    return {"world": world, "shard_rows": S, "ms_per_step_one_gpu_emulation": ms,
-            "steps": K, "warmup": W,
-            "indices_and_pool_equal_one_device": bool(same),
-            "out_rel_l2_vs_one_device": err,
-            "note": (f"{world} shards of every sequence run back to back on one GPU, each "
-                     "exchange a device copy; the time is the sum over shards plus the "
-                     "replicated merges, not a multi-GPU step time")}
+
+    def timed(run):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for i in range(K):
+            flush_l2()
+            ev[i][0].record(stream)
+            run()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(x.elapsed_time(y) for x, y in ev) / K
+
+    ms_direct = timed(step)
+    # the same step as one CUDA graph: the shards' launches without Python in between
+    ms_graph, graph_note = None, None
+    try:
+        ref = [r.idx.clone() for r in ranks]
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        for r in ranks:
+            r.idx.fill_(-9)
+        graph.replay()
+        torch.cuda.synchronize()
+        if all(torch.equal(r.idx, x) for r, x in zip(ranks, ref)):
+            ms_graph = timed(graph.replay)
+        else:
+            graph_note = "graph replay differs from direct launches"
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        torch.cuda.synchronize()
+        graph_note = f"{type(exc).__name__}: {exc}"[:200]
+    # this library's kernel launches per shard and step (the exchanges' copies excluded)
+    modes, hsi = [int(m) for m in wl.modes], wl.pool_blocks > 0
+    per_shard = 1 + wl.L + 3
+    for l, m in enumerate(modes):
+        if m == 2 or (m == 1 and hsi):
+            continue
+        jobs = 1
+        if hsi and m == 0:
+            for x in modes[l + 1:]:
+                if x == 0:
+                    break
+                jobs += x == 1
+        per_shard += 3 + (1 if wl.B > 1 and world > 1 else 0) + 3 * jobs
+    out = {"world": world, "shard_rows": S, "ms_per_step_one_gpu_emulation": ms_direct,
+           "ms_per_step_one_gpu_emulation_graph": ms_graph,
+           "launches_per_shard": per_shard, "steps": K, "warmup": W,
+           "indices_and_pool_equal_one_device": bool(same),
+           "out_rel_l2_vs_one_device": err,
+           "note": (f"{world} shards of every sequence run back to back on one GPU, each "
+                    "exchange a device copy; the time is the sum over shards plus the "
+                    "replicated merges, not a multi-GPU step time; the first figure launches "
+                    "from Python, the second replays the step as one CUDA graph")}
+    if graph_note:
+        out["graph"] = graph_note
+    return out
 
 
 def run_gpu(args, wl, rank, world):
