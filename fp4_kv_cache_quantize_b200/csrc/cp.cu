@@ -31,6 +31,8 @@
 // it exchanges are bit-identical to those the local selection ranked.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "csa2_internal.cuh"
 #include "kernels.h"
 #include "select.cuh"
@@ -40,6 +42,8 @@ namespace csa2 {
 // ----------------------------------------------------------- shard sizes
 __global__ void cp_local_rows_kernel(const int32_t* n_rows, int32_t batch, int64_t lo,
                                      int32_t shard_rows, int32_t* local_rows, uint32_t* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
     const int n = n_rows[b];
     if (n < 0) set_status(status, ST_DEVICE_CHECK);
@@ -51,6 +55,8 @@ __global__ void cp_local_rows_kernel(const int32_t* n_rows, int32_t batch, int64
 // [world][B][nb] -> [B][world * nb]: sequence b's block maxima in global block order.
 __global__ void cp_bm_regroup_kernel(const float* __restrict__ src, int32_t world, int32_t batch,
                                      int32_t nb, float* __restrict__ dst) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t per_seq = (int64_t)world * nb, total = per_seq * batch;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -68,6 +74,8 @@ constexpr int CPF_NT = 256;
 
 __global__ void __launch_bounds__(CPF_NT) cp_filter_kernel(const CpFilterParams p) {
   __shared__ uint32_t wsum[32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.x, t = threadIdx.x;
   int n = p.count[b];
   if (n < 0 || n > p.stride) {
@@ -134,6 +142,8 @@ constexpr int CPX_NT = 256;
 constexpr int CPX_ROWS = CPX_NT / 32 * 16;  // rows per CTA
 
 __global__ void __launch_bounds__(CPX_NT) cp_export_kernel(const CpExportParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int c = lane & 3, grp = lane >> 2;
   int n = p.idx_count[b];
@@ -221,6 +231,8 @@ struct CpMergeSmem {
 __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergeParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   CpMergeSmem& sm = *reinterpret_cast<CpMergeSmem*>(smem_raw);
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.x, t = threadIdx.x;
   const int n = p.world * p.top_k;  // <= CPM_NT * CPM_KPT, checked by the host
   uint32_t key[CPM_KPT];
@@ -253,6 +265,8 @@ __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergePa
 // (O, max, sum) in the same form.
 template <bool FINAL>
 __global__ void __launch_bounds__(128) cp_attn_merge_kernel(const CpAttnMergeParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int h = blockIdx.x, b = blockIdx.y, li = blockIdx.z;
   const int t = threadIdx.x, np = p.nparts;
   const int64_t slot = (int64_t)li * p.batch + b;
@@ -312,12 +326,30 @@ __global__ void __launch_bounds__(128) cp_attn_merge_kernel(const CpAttnMergePar
 }
 
 // --------------------------------------------------------------- launchers
+// Every kernel here starts with griddepcontrol.launch_dependents + .wait and is
+// launched with programmatic stream serialisation, like the rest of the
+// library, so a chain of them overlaps each launch with its predecessor's tail.
+template <typename... P, typename... A>
+static cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, A&&... args) {
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 cudaError_t launch_cp_local_rows(const int32_t* n_rows, int batch, int64_t lo, int shard_rows,
                                  int32_t* local_rows, uint32_t* status, cudaStream_t st) {
   trace_mark("cp_local_rows", st);
-  cp_local_rows_kernel<<<(batch + 255) / 256, 256, 0, st>>>(n_rows, batch, lo, shard_rows,
-                                                             local_rows, status);
-  return cudaGetLastError();
+  return launch_pdl(cp_local_rows_kernel, dim3((batch + 255) / 256), dim3(256), 0, st, n_rows,
+                    (int32_t)batch, lo, (int32_t)shard_rows, local_rows, status);
 }
 
 cudaError_t launch_cp_bm_regroup(const float* src, int world, int batch, int nb, float* dst,
@@ -327,20 +359,19 @@ cudaError_t launch_cp_bm_regroup(const float* src, int world, int batch, int nb,
   if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
   if (blocks < 1) blocks = 1;
   trace_mark("cp_bm_regroup", st);
-  cp_bm_regroup_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, world, batch, nb, dst);
-  return cudaGetLastError();
+  return launch_pdl(cp_bm_regroup_kernel, dim3((unsigned)blocks), dim3(256), 0, st, src,
+                    (int32_t)world, (int32_t)batch, (int32_t)nb, dst);
 }
 
 cudaError_t launch_cp_filter(const CpFilterParams& p, int batch, cudaStream_t st) {
   trace_mark("cp_filter", st);
-  cp_filter_kernel<<<batch, CPF_NT, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(cp_filter_kernel, dim3(batch), dim3(CPF_NT), 0, st, p);
 }
 
 cudaError_t launch_cp_export(const CpExportParams& p, int batch, cudaStream_t st) {
   trace_mark("cp_export", st);
-  cp_export_kernel<<<dim3((p.top_k + CPX_ROWS - 1) / CPX_ROWS, batch), CPX_NT, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(cp_export_kernel, dim3((p.top_k + CPX_ROWS - 1) / CPX_ROWS, batch),
+                    dim3(CPX_NT), 0, st, p);
 }
 
 cudaError_t launch_cp_merge_select(const CpMergeParams& p, cudaStream_t st) {
@@ -352,19 +383,16 @@ cudaError_t launch_cp_merge_select(const CpMergeParams& p, cudaStream_t st) {
   });
   if (ea != cudaSuccess) return ea;
   trace_mark("cp_merge_select", st);
-  cp_merge_select_kernel<<<p.batch, CPM_NT, sizeof(CpMergeSmem), st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(cp_merge_select_kernel, dim3(p.batch), dim3(CPM_NT), sizeof(CpMergeSmem), st,
+                    p);
 }
 
 cudaError_t launch_cp_attn_merge(const CpAttnMergeParams& p, int n_layers, bool final_out,
                                  cudaStream_t st) {
   const dim3 grid(CSA2_H, p.batch, n_layers);
   trace_mark(final_out ? "cp_attn_combine" : "cp_attn_local_merge", st);
-  if (final_out)
-    cp_attn_merge_kernel<true><<<grid, 128, 0, st>>>(p);
-  else
-    cp_attn_merge_kernel<false><<<grid, 128, 0, st>>>(p);
-  return cudaGetLastError();
+  if (final_out) return launch_pdl(cp_attn_merge_kernel<true>, grid, dim3(128), 0, st, p);
+  return launch_pdl(cp_attn_merge_kernel<false>, grid, dim3(128), 0, st, p);
 }
 
 int cp_merge_capacity() { return CPM_NT * CPM_KPT; }
