@@ -14,6 +14,11 @@ Timing: CUDA events on the launching stream around every step, L2 flushed
 ranks.  --gpus N > 1 runs N independent replicas (the decode step has no
 exchange to make across GPUs), one per rank, launched by torchrun.
 The reference arm (--impl reference) times the CPU oracle on the host cores.
+
+Beside the headline step the line carries, under "next_rows", the cache-append
+call, a 4-query (draft verification) step, a 64-token prefill chunk, and the
+context-parallel step with every sequence cut into 8 shards run on this one
+GPU (checked against the one-device step's indices, pool and output).
 """
 from __future__ import annotations
 
