@@ -383,6 +383,98 @@ def time_multi_query(csa2, wl, kv, dev, stream, flush_l2, K, W, with_cpu, Q=4):
     return out
 
 
+def time_layer_sequential(csa2, wl, kv, bufs, grp, stream, flush_l2, K, W):
+    """The same layer group as a layer-sequential schedule: each layer's index
+    step (csa2_index_full / csa2_index_reindex) and attention
+    (csa2_sparse_attn_decode) run after the previous layer's, as a decoder whose
+    queries come from the previous layer would run them.  Timed like the
+    headline (one CUDA graph per step when capture works, L2 flushed between
+    steps); its indices must equal the grouped step's."""
+    import torch
+    q_idx, w_h, q, swa, swa_len = bufs
+    dev = q.device
+    L, B, Kk, P = wl.L, wl.B, wl.top_k, wl.pool_blocks
+    modes = [int(m) for m in wl.modes]
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx = torch.full((L, B, Kk), -1, **i32)
+    # per-layer counts on 16-byte boundaries (the entry points' alignment rule)
+    cnt_rows = torch.zeros((L, (B + 3) // 4 * 4), **i32)
+    cnt = [cnt_rows[l, :B] for l in range(L)]
+    pool = torch.full((B, max(P, 1)), -1, **i32)
+    pcnt = torch.zeros((B,), **i32)
+    out = torch.zeros((L, B, 16, 512), dtype=torch.bfloat16, device=dev)
+    ws_i = csa2.workspace(csa2.csa2_index_workspace_size(kv, Kk, P), device=dev)
+    ws_a = csa2.workspace(csa2.csa2_attn_workspace_size(B, 1), device=dev)
+    sm = csa2.D ** -0.5
+
+    def step():
+        src = 0
+        for l, m in enumerate(modes):
+            if m == 0:
+                csa2.csa2_index_full(kv, q_idx[l], w_h[l], Kk, P, idx[l], cnt[l],
+                                     pool if P else None, pcnt if P else None, ws_i)
+                src = l
+            elif m == 1:
+                csa2.csa2_index_reindex(kv, q_idx[l], w_h[l], pool if P else None,
+                                        pcnt if P else None, max(P, 1), Kk, idx[l], cnt[l], ws_i)
+                src = l
+            csa2.csa2_sparse_attn_decode(q[l], kv, idx[src], cnt[src], Kk, swa[l], swa_len, sm,
+                                         out[l], ws_a)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    csa2.csa2_sync_status(ws_i)
+    csa2.csa2_sync_status(ws_a)
+    # REUSE layers of the grouped step hold copies of their source's indices
+    src_of, src = [], 0
+    for l, m in enumerate(modes):
+        src = l if m != 2 else src
+        src_of.append(src)
+    same = all(torch.equal(idx[src_of[l]], grp.idx[l]) and torch.equal(cnt[src_of[l]],
+                                                                        grp.idx_count[l])
+               for l in range(L))
+    a, b = out.double(), grp.out.double()
+    err = float((a - b).norm() / max(float(b.norm()), 1e-30))
+
+    def timed(run):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for i in range(K):
+            flush_l2()
+            ev[i][0].record(stream)
+            run()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return sorted(x.elapsed_time(y) for x, y in ev)
+
+    launch, times = "direct", None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        ref = idx.clone()
+        idx.fill_(-9)
+        graph.replay()
+        torch.cuda.synchronize()
+        if torch.equal(idx, ref):
+            times, launch = timed(graph.replay), "cuda_graph"
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        torch.cuda.synchronize()
+        launch = f"direct ({type(exc).__name__}: {exc})"[:200]
+    if times is None:
+        times = timed(step)
+    ms = statistics.median(times)
+    return {"ms_per_step": ms, "value": B * L / (ms * 1e-3), "unit": "layer-steps/s",
+            "step_launch": launch, "steps": K, "warmup": W,
+            "indices_equal_grouped_step": bool(same), "out_rel_l2_vs_grouped_step": err,
+            "note": ("context row: every layer's index step and attention after the previous "
+                     "layer's (csa2_index_full / csa2_index_reindex / csa2_sparse_attn_decode "
+                     "per layer); the headline groups them (one scan + select DAG, one "
+                     "attention launch for all layers)")}
+
+
 def time_context_parallel(csa2, wl, bufs, grp, stream, flush_l2, K, W, world=8):
     """The context-parallel decode step with every sequence cut into `world`
     shards, all run on this one GPU (LocalComm: the shards' kernels back to
@@ -683,6 +775,12 @@ def run_gpu(args, wl, rank, world):
     prefill["note"] = ("chunked prefill of 64 new tokens; the scan runs 8 passes of 8 queries "
                        "(MMA N = 64)")
     try:
+        seq = time_layer_sequential(csa2, wl, kv, (q_idx, w_h, q, swa, swa_len), grp, stream,
+                                    flush_l2, 20, 3)
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        torch.cuda.synchronize()
+        seq = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+    try:
         cpar = time_context_parallel(
             csa2, wl, (codes, scales, idxk, n_rows, pt, q_idx, w_h, q, swa, swa_len), grp, stream,
             flush_l2, 10, 3)
@@ -725,6 +823,7 @@ def run_gpu(args, wl, rank, world):
                                "output, indices) copied back, on separate streams overlapping "
                                "the neighbouring steps' compute; no L2 flush (134 MB of "
                                "indexer K per step exceeds the 126 MB L2)")},
+            "layer_sequential": seq,
             "next_rows": {"cache_append": append, "multi_query": multi,
                           "prefill_chunk": prefill, "context_parallel": cpar},
             "gpu_launches": int(launches * K),
