@@ -774,19 +774,26 @@ def run_gpu(args, wl, rank, world):
     prefill = time_multi_query(csa2, wl, kv, dev, stream, flush_l2, 5, 3, with_cpu, Q=64)
     prefill["note"] = ("chunked prefill of 64 new tokens; the scan runs 8 passes of 8 queries "
                        "(MMA N = 64)")
+    def quiet_sync():
+        # a failed optional measurement must not take the headline line with it
+        try:
+            torch.cuda.synchronize()
+        except Exception:  # noqa: BLE001
+            pass
+
     try:
         seq = time_layer_sequential(csa2, wl, kv, (q_idx, w_h, q, swa, swa_len), grp, stream,
                                     flush_l2, 20, 3)
     except Exception as exc:  # noqa: BLE001  (reported in the line)
-        torch.cuda.synchronize()
         seq = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        quiet_sync()
     try:
         cpar = time_context_parallel(
             csa2, wl, (codes, scales, idxk, n_rows, pt, q_idx, w_h, q, swa, swa_len), grp, stream,
             flush_l2, 10, 3)
     except Exception as exc:  # noqa: BLE001  (reported in the line)
-        torch.cuda.synchronize()
         cpar = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        quiet_sync()
 
     units = wl.B * wl.L
     value = job_throughput(units, world, t_step)
