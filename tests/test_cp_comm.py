@@ -74,3 +74,17 @@ def test_local_comm_rejects_a_missing_shard():
     from fp4_kv_cache_quantize_b200 import cp
     with pytest.raises(ValueError):
         cp.LocalComm(3).all_gather([torch.zeros(2), torch.zeros(2)])
+
+
+def test_local_view_checks_the_layout():
+    from fp4_kv_cache_quantize_b200 import cp
+    codes = torch.zeros((1024, 256), dtype=torch.uint8)
+    scales = torch.zeros((1024, 32), dtype=torch.uint8)
+    k = torch.zeros((1024, 64), dtype=torch.int16)
+    with pytest.raises(ValueError, match="seq_stride"):
+        cp.local_view(codes, scales, k, rank=0, world=4, shard_rows=256, batch=2, seq_stride=512)
+    with pytest.raises(ValueError, match="64-row page"):
+        cp.local_view(codes, scales, k, rank=0, world=2, shard_rows=96, batch=1,
+                      page_table=torch.zeros((1, 4), dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA device"):   # the binding takes device tensors only
+        cp.local_view(codes, scales, k, rank=1, world=2, shard_rows=256, batch=2, seq_stride=512)
