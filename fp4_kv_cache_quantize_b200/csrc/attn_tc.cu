@@ -1,0 +1,524 @@
+// attn_tc.cu -- sparse + sliding-window decode attention on the tensor cores.
+//
+// For one (layer, sequence): keys = values = [the Top-k main-KV rows, FP4
+// dequantised exactly ; the layer's 128-row E4M3 window], one softmax over
+// both branches, 16 query heads sharing every row (tucaod.com walk-through,
+// core-attention figure: selection, Top-K and concatenation of main KV and
+// SWA; release note, section "Causal Encoder-Decoder": 128-token SWA at every
+// layer; section "FP4 KV": FP8 window KV).
+//
+// One thread-block cluster of five CTAs per (layer, sequence): CTA c < 4
+// takes keys [128 c, 128 c + 128) of the sparse branch, CTA 4 the window.
+// With 16 heads a per-CTA tile is too narrow for the tensor core's 128-row
+// MMA in its natural orientation, so both products run transposed, keys and
+// channels on the MMA's M axis and the heads on N (tcgen05.mma, M = 128,
+// N = 16, fp32 accumulators in tensor memory):
+//   S^T[key][head]  = K[key][:] . Q'[head][:]       (K-major A and B)
+//   O^T[chan][head] = V^T[chan][key] . P^T[head][key] (A read MN-major from
+//                                                     the same K = V tile)
+// Every operand is fp16: E2M1 x E4M3 products and E4M3 window values are
+// exact in fp16, and each query head is scaled by a power of two (undone on
+// its logits) so that any bf16 query is represented to fp16 precision
+// without overflow.  Rows are gathered with cp.async (16 bytes per copy)
+// into shared memory and dequantised there into the 128-byte-swizzled tile
+// the MMA reads.  The softmax runs on the S^T accumulator (one thread per
+// key); P^T in fp16 is the second MMA's B operand.  The five partial results
+// (normalised O in fp16, max and sum per head) are pushed through
+// distributed shared memory to the CTA owning each 128-channel block, one
+// cluster barrier, and the owners merge them with log-sum-exp weights and
+// write the bf16 output: no partials go through global memory.
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+
+#include "csa2_internal.cuh"
+#include "kernels.h"
+
+namespace csa2 {
+
+namespace cg = cooperative_groups;
+
+constexpr int TA_NT = 256;
+constexpr int TA_KEYS = 128;                        // keys per CTA: the MMA's M
+constexpr int TA_SPARSE = CSA2_MAX_TOPK / TA_KEYS;  // CTAs of the sparse branch
+constexpr int TA_CTAS = TA_SPARSE + 1;              // and the window's
+static_assert(CSA2_W == TA_KEYS, "one CTA holds the whole window");
+constexpr int TA_KB = TA_KEYS * 128;                // one 64-channel block of the tile
+constexpr int TA_CODE_LD = 272;                     // padded shared-memory row strides
+constexpr int TA_SCALE_LD = 48;
+constexpr int TA_WIN_LD = 528;
+constexpr int TA_SCALE_OFF = TA_KEYS * TA_CODE_LD;
+constexpr int TA_RECV_OFF = TA_SCALE_OFF + TA_KEYS * TA_SCALE_LD;
+constexpr int TA_RAW_BYTES = TA_KEYS * TA_WIN_LD;
+static_assert(TA_RECV_OFF + TA_CTAS * 128 * CSA2_H * 2 <= TA_RAW_BYTES, "receive buffer");
+constexpr uint32_t TA_IDESC_QK = idesc_f16_f32(128, 16, false);
+constexpr uint32_t TA_IDESC_PV = idesc_f16_f32(128, 16, true);
+constexpr uint32_t TA_TMEM_COLS = 128;  // S^T in columns [0, 16), O^T in [64, 128)
+constexpr uint32_t TA_O_COL = 64;
+
+struct TaSmem {
+  // K = V in fp16: channel block kb at kb * TA_KB, 128 rows (keys) of 128 B,
+  // 16-byte chunks swizzled by row % 8
+  alignas(1024) uint8_t tile[8 * TA_KB];
+  alignas(1024) uint8_t q[8 * 2048];       // Q': channel block kb, 16 rows (heads) of 128 B
+  alignas(1024) uint8_t p[2 * 2048];       // P^T: key block kb, 16 rows (heads) of 128 B
+  // gathered rows: the window's E4M3 rows, or FP4 codes | scales | the
+  // normalised partials this CTA receives as the owner of a channel block
+  alignas(16) uint8_t raw[TA_RAW_BYTES];
+  int64_t row[TA_KEYS];
+  float scl1[CSA2_H], scl2[CSA2_H];        // logit = acc * scl1 * scl2 (log2 units)
+  uint32_t qmax[TA_NT / 32][4];
+  float wmax[4][CSA2_H];
+  float m[CSA2_H], lsum[CSA2_H];
+  float2 ml[TA_CTAS][CSA2_H];              // (max, sum) per source CTA, at the owners
+  float wts[TA_CTAS][CSA2_H];
+  uint64_t mbar;
+  uint32_t tmem_base;
+};
+constexpr size_t TA_SMEM = sizeof(TaSmem) + 1024;
+
+__device__ __forceinline__ int64_t ta_kv_row(const AttnParams& p, int b, int pos) {
+  if (p.page_table) {
+    const int page = pos >> 6;
+    const int64_t pid =
+        page < p.max_pages ? (int64_t)p.page_table[(int64_t)b * p.max_pages + page] : -1;
+    const int64_t row = pid * 64 + (pos & 63);
+    return (pid < 0 || row >= p.pool_rows) ? -1 : row;
+  }
+  const int64_t row = (int64_t)b * p.seq_stride + pos;
+  return row < p.pool_rows ? row : -1;
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// 2^e as a float, e in [-126, 127]
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// Byte offset of 16-byte chunk cc (0..7) of row r in a 128-byte-swizzled block.
+__device__ __forceinline__ uint32_t sw_off(int r, int cc) {
+  return (uint32_t)(r * 128 + ((cc ^ (r & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  TaSmem& s = *reinterpret_cast<TaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
+  cg::cluster_group cluster = cg::this_cluster();
+  const int c = (int)cluster.block_rank();
+  const bool window = c == TA_SPARSE;
+  const int b = blockIdx.y, li = blockIdx.z;
+  const AttnLayer L = p.layer[li];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  pdl_launch_dependents();
+
+  if (t == 0) {
+    mbar_init(&s.mbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem_base, TA_TMEM_COLS);
+    tmem_relinquish();
+  }
+
+  // ---- Q' = Q * 2^e_h in fp16: max |Q'_h| in [2^14, 2^15).  The queries
+  // are inputs (no kernel of this library writes them): read before the wait.
+  uint4 qv[4];
+  {
+    const uint4* qg = reinterpret_cast<const uint4*>(L.q + (int64_t)b * CSA2_H * CSA2_D);
+#pragma unroll
+    for (int u = 0; u < 4; u++) {  // chunk t + 256 u: head (t >> 6) + 4 u, chunk t & 63
+      qv[u] = __ldg(qg + t + TA_NT * u);
+      const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+      uint32_t mx = 0u;
+#pragma unroll
+      for (int k = 0; k < 4; k++) mx = max(mx, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+      mx = __reduce_max_sync(0xffffffffu, mx);
+      if (lane == 0) s.qmax[warp][u] = mx;
+    }
+  }
+  __syncthreads();
+  {
+    const int hq = t >> 6, cfull = t & 63, kb = cfull >> 3, cc = cfull & 7;
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+      const int h = hq + 4 * u;
+      const uint32_t mb = max(s.qmax[warp][u], s.qmax[warp ^ 1][u]);
+      const float M = __uint_as_float(mb << 16);
+      int e = 0;
+      if (M > 0.0f && M <= 3.3895314e38f) {  // finite, nonzero: 2^14 <= M 2^e < 2^15
+        int ex;
+        frexpf(M, &ex);
+        e = 15 - ex;
+      }
+      const int e1 = e / 2, e2 = e - e1;  // each within a float's exponent range
+      const float f1 = pow2i(e1), f2 = pow2i(e2);
+      if (cfull == 0) {
+        s.scl1[h] = pow2i(-e1);
+        s.scl2[h] = p.scale_log2 * pow2i(-e2);
+      }
+      const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        const float lo = __uint_as_float(w[k] << 16) * f1 * f2;
+        const float hi = __uint_as_float(w[k] & 0xFFFF0000u) * f1 * f2;
+        o4[k] = h2u(__floats2half2_rn(lo, hi));
+      }
+      *reinterpret_cast<uint4*>(s.q + kb * 2048 + sw_off(h, cc)) =
+          make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  pdl_wait();  // the indices come from the previous kernel
+
+  // ---- this CTA's keys.  b runs over sequences x queries: query tq of
+  // sequence bp sees the sequence's entries minus the drafts after it, and
+  // the window rows that end at its own entry.
+  const int bp = b / p.nq, tq = b - bp * p.nq, later = p.nq - 1 - tq;
+  int C = p.n_rows[bp];
+  if (C < 0 || C > p.max_rows) {
+    if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
+    C = C < 0 ? 0 : p.max_rows;
+  }
+  C = C - later < 0 ? 0 : C - later;
+  int nk;  // candidate keys of this CTA: keys j < nk
+  if (!window) {
+    int n_idx = L.idx_count[b];
+    if (n_idx < 0 || n_idx > p.idx_stride) {
+      if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
+      n_idx = n_idx < 0 ? 0 : p.idx_stride;
+    }
+    const int k0 = c * TA_KEYS;
+    nk = min(max(n_idx - k0, 0), TA_KEYS);
+    const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
+    if (L.idx_copy) {  // Reuse layer: publish the indices it used
+      for (int i = t; i < TA_KEYS && k0 + i < p.idx_stride; i += TA_NT)
+        L.idx_copy[(int64_t)b * p.idx_stride + k0 + i] = idx[k0 + i];
+      if (c == 0 && t == 0) L.idx_copy_count[b] = L.idx_count[b];
+    }
+    if (t < TA_KEYS) {
+      int64_t row = -1;
+      if (t < nk) {
+        const int pos = __ldg(idx + k0 + t);
+        if (pos >= 0 && pos < C) row = ta_kv_row(p, bp, pos);
+        if (row < 0) set_status(p.status, ST_DEVICE_CHECK);
+      }
+      s.row[t] = row;
+    }
+  } else {
+    int n_win = p.swa_len[bp];
+    if (n_win < 0 || n_win > p.swa_rows) {
+      if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
+      n_win = n_win < 0 ? 0 : p.swa_rows;
+    }
+    const int win_end = n_win - later < 0 ? 0 : n_win - later;
+    const int win_lo = win_end > CSA2_W ? win_end - CSA2_W : 0;
+    nk = win_end - win_lo;
+    if (t < TA_KEYS) s.row[t] = t < nk ? (int64_t)(win_lo + t) : -1;
+  }
+  __syncthreads();
+
+  // ---- gather the rows (16-byte asynchronous copies)
+  if (nk > 0) {
+    if (!window) {
+#pragma unroll
+      for (int u = 0; u < (TA_KEYS * 18 + TA_NT - 1) / TA_NT; u++) {
+        const int i = t + TA_NT * u;
+        const int r = i / 18, part = i - 18 * r;
+        if (r < TA_KEYS) {
+          const int64_t row = s.row[r];
+          if (row >= 0) {
+            if (part < 16)
+              cp_async16(s.raw + r * TA_CODE_LD + 16 * part, p.codes + row * (CSA2_D / 2) + 16 * part);
+            else
+              cp_async16(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * (part - 16),
+                         p.scales + row * (CSA2_D / 16) + 16 * (part - 16));
+          }
+        }
+      }
+    } else {
+      const uint8_t* swa = L.swa + (int64_t)bp * p.swa_rows * CSA2_D;
+#pragma unroll 4
+      for (int u = 0; u < TA_KEYS * 32 / TA_NT; u++) {
+        const int i = t + TA_NT * u, r = i >> 5, part = i & 31;
+        const int64_t row = s.row[r];
+        if (row >= 0) cp_async16(s.raw + r * TA_WIN_LD + 16 * part, swa + row * CSA2_D + 16 * part);
+      }
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+  }
+  __syncthreads();
+
+  // ---- dequantise into the fp16 tile: two threads per row, 256 channels each
+  if (nk > 0) {
+    const int r = t & (TA_KEYS - 1), half = t >> 7;
+    const bool valid = s.row[r] >= 0;
+    uint8_t* trow = s.tile;
+    if (!valid) {
+#pragma unroll
+      for (int j = 0; j < 32; j++) {
+        const int kb = 4 * half + (j >> 3), cc = j & 7;
+        *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc)) = make_uint4(0, 0, 0, 0);
+      }
+    } else if (!window) {
+      const uint8_t* cr = s.raw + r * TA_CODE_LD + 128 * half;
+      const uint4 sc = *reinterpret_cast<const uint4*>(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD +
+                                                       16 * half);
+      const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+      for (int i = 0; i < 8; i++) {  // 16 code bytes: channels 256 half + 32 i + [0, 32)
+        const uint4 cv = *reinterpret_cast<const uint4*>(cr + 16 * i);
+        const uint32_t words[4] = {cv.x, cv.y, cv.z, cv.w};
+        const uint32_t sb = (scw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;  // groups 2i, 2i+1
+        const __half s0 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sb & 0xFF), __NV_E4M3));
+        const __half s1 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sb >> 8), __NV_E4M3));
+        const int kb = 4 * half + (i >> 1);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; q4++) {  // 8 channels per 16-byte store
+          const uint32_t word = words[q4];
+          const __half2 scv = q4 < 2 ? __half2(s0, s0) : __half2(s1, s1);
+          uint32_t hv[4];
+#pragma unroll
+          for (int k = 0; k < 4; k++)
+            hv[k] = h2u(__hmul2(__half2(__nv_cvt_fp4x2_to_halfraw2(
+                                    (__nv_fp4x2_storage_t)((word >> (8 * k)) & 0xFF), __NV_E2M1)),
+                                scv));
+          const int cc = 4 * (i & 1) + q4;
+          *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc)) =
+              make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        }
+      }
+    } else {
+      const uint8_t* wr = s.raw + r * TA_WIN_LD + 256 * half;
+#pragma unroll
+      for (int j = 0; j < 16; j++) {  // 16 E4M3 bytes: channels 256 half + 16 j + [0, 16)
+        const uint4 v = *reinterpret_cast<const uint4*>(wr + 16 * j);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t hv[8];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          hv[2 * k] = h2u(__half2(__nv_cvt_fp8x2_to_halfraw2(
+              (__nv_fp8x2_storage_t)(wv[k] & 0xFFFF), __NV_E4M3)));
+          hv[2 * k + 1] = h2u(__half2(__nv_cvt_fp8x2_to_halfraw2(
+              (__nv_fp8x2_storage_t)(wv[k] >> 16), __NV_E4M3)));
+        }
+        const int kb = 4 * half + (j >> 2), cc = 2 * (j & 3);
+        *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc)) =
+            make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc + 1)) =
+            make_uint4(hv[4], hv[5], hv[6], hv[7]);
+      }
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // ---- S^T = K . Q'^T (one thread issues 32 MMAs of K = 16)
+  if (nk > 0 && t == 0) {
+    tc_fence_after();
+    const uint32_t a0 = smem_u32(s.tile), b0 = smem_u32(s.q);
+#pragma unroll
+    for (int kb = 0; kb < 8; kb++)
+#pragma unroll
+      for (int sub = 0; sub < 4; sub++)
+        umma_bf16(tmem, sdesc_k128(a0 + kb * TA_KB + 32 * sub), sdesc_k128(b0 + kb * 2048 + 32 * sub),
+                  TA_IDESC_QK, (kb | sub) != 0);
+    umma_commit(&s.mbar);
+  }
+  bool ok = true;
+  if (nk > 0 && warp < 4) {
+    // ---- softmax over this CTA's keys: thread = key, 16 heads
+    ok = __all_sync(0xffffffffu, mbar_wait(&s.mbar, 0, nullptr));
+    if (!ok && lane == 0) set_status(p.status, ST_TIMEOUT);
+    tc_fence_after();
+    uint32_t r[16];
+    tmem_ld_x16(tmem + ((uint32_t)(32 * warp) << 16), r);
+    tmem_ld_wait();
+    const int key = 32 * warp + lane;
+    const bool valid = ok && key < nk && s.row[key] >= 0;
+    float x[16];
+#pragma unroll
+    for (int h = 0; h < 16; h++) {
+      x[h] = valid ? __uint_as_float(r[h]) * s.scl1[h] * s.scl2[h] : -INFINITY;
+      const float mh = warp_max_f32(x[h]);
+      if (lane == h) s.wmax[warp][h] = mh;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int kb = key >> 6, cc = (key & 63) >> 3;
+#pragma unroll
+    for (int h = 0; h < 16; h++) {
+      const float m = fmaxf(fmaxf(s.wmax[0][h], s.wmax[1][h]), fmaxf(s.wmax[2][h], s.wmax[3][h]));
+      const float pe = m == -INFINITY ? 0.0f : exp2f(x[h] - m);
+      *reinterpret_cast<__half*>(s.p + kb * 2048 + sw_off(h, cc) + (key & 7) * 2) = __float2half_rn(pe);
+      if (lane == h && warp == 0) s.m[h] = m;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // ---- O^T = V^T . P^T: four channel blocks of 128, K = 128 keys in 8 steps
+  if (nk > 0 && t == 0) {
+    tc_fence_after();
+    const uint32_t a0 = smem_u32(s.tile), b0 = smem_u32(s.p);
+#pragma unroll
+    for (int cb = 0; cb < 4; cb++)
+#pragma unroll
+      for (int ks = 0; ks < 8; ks++)
+        umma_bf16(tmem + TA_O_COL + 16 * cb,
+                  sdesc_mn128(a0 + cb * 2 * TA_KB + ks * 2048, TA_KB, 1024),
+                  sdesc_k128(b0 + (ks >> 2) * 2048 + (ks & 3) * 32), TA_IDESC_PV, ks > 0);
+    umma_commit(&s.mbar);
+  }
+  if (warp >= 4) {
+    // ---- the softmax sums from the fp16 probabilities the MMA reads:
+    // 8 threads per head, 16 keys each
+    const int u = t - 128, h = u >> 3, seg = u & 7;
+    float l = 0.0f;
+    if (nk > 0) {
+#pragma unroll
+      for (int k2 = 0; k2 < 2; k2++) {
+        const int cc = 2 * (seg & 3) + k2;
+        const uint4 v = *reinterpret_cast<const uint4*>(s.p + (seg >> 2) * 2048 + sw_off(h, cc));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+          l += f.x + f.y;
+        }
+      }
+    }
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    if (seg == 0) s.lsum[h] = l;
+  }
+  if (nk == 0 && t < CSA2_H) s.m[t] = -INFINITY;
+  __syncthreads();
+
+  // ---- normalised partial O^T -> the owners of the channel blocks
+  if (warp < 4) {
+    uint32_t o[4][16];
+    bool ok2 = ok;
+    if (nk > 0) {
+      ok2 = __all_sync(0xffffffffu, ok && mbar_wait(&s.mbar, 1, nullptr));
+      if (!ok2 && lane == 0 && ok) set_status(p.status, ST_TIMEOUT);
+      tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < 4; cb++)
+        tmem_ld_x16(tmem + ((uint32_t)(32 * warp) << 16) + TA_O_COL + 16 * cb, o[cb]);
+      tmem_ld_wait();
+    }
+    const bool live = nk > 0 && ok2;
+    if (live) {
+      float inv[16];
+#pragma unroll
+      for (int h = 0; h < 16; h++) inv[h] = s.lsum[h] > 0.0f ? 1.0f / s.lsum[h] : 0.0f;
+      const int chl = 32 * warp + lane;
+#pragma unroll
+      for (int cb = 0; cb < TA_SPARSE; cb++) {
+        uint32_t hv[8];
+#pragma unroll
+        for (int k = 0; k < 8; k++)
+          hv[k] = h2u(__floats2half2_rn(__uint_as_float(o[cb][2 * k]) * inv[2 * k],
+                                        __uint_as_float(o[cb][2 * k + 1]) * inv[2 * k + 1]));
+        uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(
+            s.raw + TA_RECV_OFF + ((c * 128 + chl) * CSA2_H) * 2, cb));
+        dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+      }
+    }
+    if (t < CSA2_H) {
+      const float2 ml = live ? make_float2(s.m[t], s.lsum[t]) : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+      for (int o2 = 0; o2 < TA_SPARSE; o2++) *cluster.map_shared_rank(&s.ml[c][t], o2) = ml;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TA_TMEM_COLS);
+  }
+  cluster.sync();  // every partial has arrived; no remote access after this
+
+  // ---- owners: log-sum-exp merge of the five partials of 128 channels
+  if (c < TA_SPARSE) {
+    if (t < CSA2_H) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int src = 0; src < TA_CTAS; src++) M = fmaxf(M, s.ml[src][t].x);
+      float Lsum = 0.0f, wv[TA_CTAS];
+#pragma unroll
+      for (int src = 0; src < TA_CTAS; src++) {
+        const float2 ml = s.ml[src][t];
+        wv[src] = ml.x == -INFINITY ? 0.0f : ml.y * exp2f(ml.x - M);
+        Lsum += wv[src];
+      }
+      const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+#pragma unroll
+      for (int src = 0; src < TA_CTAS; src++) s.wts[src][t] = wv[src] * inv;
+    }
+    __syncthreads();
+    if (t < 128) {
+      float acc[16];
+#pragma unroll
+      for (int h = 0; h < 16; h++) acc[h] = 0.0f;
+#pragma unroll
+      for (int src = 0; src < TA_CTAS; src++) {
+        const uint4* v =
+            reinterpret_cast<const uint4*>(s.raw + TA_RECV_OFF + ((src * 128 + t) * CSA2_H) * 2);
+        const uint4 v0 = v[0], v1 = v[1];
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          const float wa = s.wts[src][2 * k], wb = s.wts[src][2 * k + 1];
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+          if (wa != 0.0f) acc[2 * k] = fmaf(wa, f.x, acc[2 * k]);
+          if (wb != 0.0f) acc[2 * k + 1] = fmaf(wb, f.y, acc[2 * k + 1]);
+        }
+      }
+      uint16_t* out = L.out + (int64_t)b * CSA2_H * CSA2_D + c * 128 + t;
+#pragma unroll
+      for (int h = 0; h < 16; h++) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(acc[h]);
+        out[h * CSA2_D] = *reinterpret_cast<const uint16_t*>(&v);
+      }
+    }
+  }
+}
+
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t st) {
+  static PerDeviceOnce attr;
+  cudaError_t ea = attr.run([](int&) {
+    return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)TA_SMEM);
+  });
+  if (ea != cudaSuccess) return ea;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = TA_CTAS;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(TA_CTAS, p.batch, p.n_layers);
+  cfg.blockDim = dim3(TA_NT);
+  cfg.dynamicSmemBytes = TA_SMEM;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  trace_mark("attn", st);
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, p);
+}
+
+}  // namespace csa2

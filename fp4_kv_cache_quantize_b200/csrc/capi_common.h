@@ -19,6 +19,9 @@ int num_sms();
 // Records the next trace event (see csa2_trace_set) before a launch.
 void trace_mark(const char* stage, cudaStream_t st);
 
+// Host-side checks of csa2_index_full's view and sizes (capi_index.cu).
+csa2_status check_index_args(const csa2_kv_view* kv, int top_k, int pool_blocks);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 #define CSA2_REQUIRE(cond, status, ...) \

@@ -99,6 +99,12 @@ static csa2_status check_topk(int top_k, int pool_blocks) {
   return CSA2_OK;
 }
 
+csa2_status check_index_args(const csa2_kv_view* kv, int top_k, int pool_blocks) {
+  csa2_status r = check_kv(kv);
+  if (r) return r;
+  return check_topk(top_k, pool_blocks);
+}
+
 // ------------------------------------------------------------ workspace
 struct IndexWs {
   uint32_t* status;
@@ -435,7 +441,7 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, const csa2_kv_view* kv, c
   ap.part_o = reinterpret_cast<float*>(base + CSA2_WS_HEADER);
   ap.part_ml = reinterpret_cast<float*>(base + CSA2_WS_HEADER + slots * CSA2_H * CSA2_D * 4);
   ap.status = static_cast<uint32_t*>(ws);
-  CSA2_CUDA(launch_attn(ap, (cudaStream_t)stream));
+  CSA2_CUDA(launch_attn_tc(ap, (cudaStream_t)stream));
   trace_mark("end", (cudaStream_t)stream);
   return CSA2_OK;
 }
@@ -539,7 +545,7 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
                             reuse ? layer_cnt(l) : nullptr,
                             d->out + (size_t)l * VB * CSA2_H * CSA2_D};
   }
-  CSA2_CUDA(launch_attn(ap, st));
+  CSA2_CUDA(launch_attn_tc(ap, st));
   trace_mark("end", st);
   return CSA2_OK;
 }

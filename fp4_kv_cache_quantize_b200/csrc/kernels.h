@@ -131,6 +131,9 @@ int attn_nsplit(int pairs, int num_sms);
 size_t attn_partial_bytes(int batch, int n_layers, int nsplit);
 // merge = false leaves the split partials in part_o / part_ml (nsplit > 1).
 cudaError_t launch_attn(const AttnParams& p, cudaStream_t st, bool merge = true);
+// The tensor-core attention: one 5-CTA cluster per (layer, sequence), merged
+// in the cluster, bf16 output (part_o / part_ml unused).
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t st);
 
 // ------------------------------------------------------------ cache append
 struct AppendParams {

@@ -14,6 +14,7 @@ Input recipe (shapes and distributions of the workloads):
   main KV x          bf16 [rows, 512], N(0,1) (optionally 0.1% of elements x50)
   indexer weights    bf16 [512, 64], N(0, 1/512)
   indexer K          bf16 [rows, 64] = bf16(x @ W_idx), fp64 sum of exact products
+                     rounded once to bf16
   indexer query      bf16 [L, B, 8, 64], N(0,1)
   indexer head w     fp32 [L, B, 8], U(0,1)
   main query         bf16 [L, B, 16, 512], N(0,1)
@@ -47,6 +48,17 @@ def rng(seed: int, stream: int, chunk: int = 0) -> np.random.Generator:
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
     t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
     return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def f64_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """bf16 bits of float64 values, rounded once to nearest-even (no float32
+    step in between): 8 significant bits below the leading one, or the
+    subnormal spacing 2^-133 below 2^-126."""
+    x = np.asarray(a, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                 # bf16 subnormals: fixed spacing 2^-133
+    r = np.ldexp(np.rint(np.ldexp(x, 8 - e)), e - 8)   # exact in float64; rint is RNE
+    return to_bf16_bits(r.astype(np.float32))          # exact: r is a bf16 value
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -128,10 +140,11 @@ class Workload:
             x[max(lo, 0):min(hi, n)] += (self.planted_beta * v).astype(np.float32)
 
     def idxk_of(self, x_bits: np.ndarray) -> np.ndarray:
-        """bf16 indexer K of bf16 main-KV rows: bf16(x @ W_idx) in fp64."""
+        """bf16 indexer K of bf16 main-KV rows: x @ W_idx summed in fp64 and
+        rounded once to bf16 (nearest even), the cache-append rule."""
         xf = bf16_bits_to_f32(x_bits).astype(np.float64)
         wf = bf16_bits_to_f32(self.w_idx).astype(np.float64)
-        return to_bf16_bits((xf @ wf).astype(np.float32))
+        return f64_to_bf16_bits(xf @ wf)
 
     def chunk(self, c: int):
         x = self.x_chunk(c)

@@ -94,3 +94,25 @@ def test_cp_host_validation(lib):
     assert m(ctypes.byref(sh), ctypes.c_void_p(260), 1, 0, 1, 512, p, p, p, 256, None) == 3
     assert m(ctypes.byref(sh), p, 1, 0, 1, 513, p, p, p, 256, None) == 2   # top_k > 512
 
+
+
+def test_noalloc_checks_arguments_before_its_scratch_size():
+    """csa2_index_full_noalloc validates the view and sizes like
+    csa2_index_full, so a bad shape reports CSA2_ERR_SHAPE rather than a
+    scratch-size error, and nothing is enqueued (no GPU here)."""
+    from fp4_kv_cache_quantize_b200 import csa2
+    lib2 = csa2._lib
+    p = ctypes.c_void_p(256)
+    kv = csa2.KVView()
+    kv.codes = kv.scales = kv.idx_k = kv.n_rows = p
+    kv.batch, kv.max_rows, kv.seq_stride, kv.pool_rows = -3, 1024, 1024, 1024
+    f = lib2.csa2_index_full_noalloc
+    args = (p, p, 512, 2048, p, p, p, p, None)
+    assert f(ctypes.byref(kv), *args) == 2          # negative batch: a shape error
+    kv.batch, kv.max_rows = 1, -5
+    assert f(ctypes.byref(kv), *args) == 2          # negative max_rows: a shape error
+    kv.max_rows = 1024
+    assert f(ctypes.byref(kv), p, p, 0, 2048, p, p, p, p, None) == 2     # top_k = 0
+    assert f(ctypes.byref(kv), p, None, 512, 2048, p, p, p, p, None) == 1  # NULL weights
+    kv.batch, kv.max_rows, kv.seq_stride, kv.pool_rows = 8, 1 << 20, 1 << 20, 8 << 20
+    assert f(ctypes.byref(kv), *args) == 4          # 8 x 1M positions: beyond the scratch

@@ -45,6 +45,33 @@ def test_projection_rounding_ties_go_to_even(orc):
     assert orc.project_idxk(x, w)[0] == bf16_bits([1 - 2.0 ** -8])[0]
 
 
+def test_synthetic_indexer_k_rounds_once_like_the_append_rule(orc):
+    """The decode inputs' indexer K (synth) follows the append path's rule:
+    the fp64 sum rounded once to bf16.  Sums that sit on a bf16 rounding
+    midpoint in fp64 but not after a float32 step tell one rounding from two."""
+    w = np.zeros((512, 64), np.uint16)
+    w[0, :] = bf16_bits([1.0])[0]
+    w[1, :] = bf16_bits([2.0 ** -8])[0]
+    w[2, :] = bf16_bits([2.0 ** -30])[0]
+    x = np.zeros((6, 512), np.uint16)
+    x[:, 0] = bf16_bits([1.0])[0]
+    x[0, 1] = bf16_bits([1.0])[0]                      # 1 + 2^-8: tie, to even (1)
+    x[1, 1], x[1, 2] = bf16_bits([1.0])[0], bf16_bits([1.0])[0]   # just above the tie
+    x[2, 1], x[2, 2] = bf16_bits([1.0])[0], bf16_bits([-1.0])[0]  # just below the tie
+    x[3, 1] = bf16_bits([3.0])[0]                      # 1 + 3 2^-8: tie, to even (1 + 2^-6)
+    x[4, 2] = bf16_bits([5.0])[0]                      # 1 + 5 2^-30: rounds to 1
+    x[5] = bf16_bits(np.random.default_rng(3).standard_normal(512))
+    wl = type("W", (), {"w_idx": w})()
+    got = synth.Workload.idxk_of(wl, x)
+    want = np.stack([orc.project_idxk(x[i], w) for i in range(len(x))])
+    assert np.array_equal(got, want)
+    # the float32 step would have moved the first "just above" and "just
+    # below" sums onto the tie (1 + 2^-8 +- 2^-30 is not a float32 value)
+    assert got[1, 0] == 0x3F81 and got[2, 0] == 0x3F80
+    assert not np.array_equal(got, synth.to_bf16_bits(
+        (bf16_vals(x) @ bf16_vals(w)).astype(np.float32)))
+
+
 def _neighbours(bits):
     return (bits.astype(np.int32) + 1).astype(np.uint16), (bits.astype(np.int32) - 1).astype(np.uint16)
 
