@@ -568,6 +568,286 @@ def time_context_parallel(csa2, wl, bufs, grp, stream, flush_l2, K, W, world=8):
     return out
 
 
+# ------------------------------------------------------------ other configs
+QUANT_BYTES_PER_ROW = 1024 + 256 + 32    # bf16 row in, FP4 codes + E4M3 scales out
+
+
+def sub_workload(wl, S: int):
+    """The first S sequences of a workload (same row pool, same seeds)."""
+    import dataclasses
+    pt = None if wl.page_table is None else np.ascontiguousarray(wl.page_table[:S])
+    sub = dataclasses.replace(wl, B=S, n_rows=wl.n_rows[:S].copy(), page_table=pt)
+    for name in ("q_idx", "w_h", "q", "swa"):
+        setattr(sub, name, np.ascontiguousarray(getattr(wl, name)[:, :S]))
+    sub.swa_len = wl.swa_len[:S].copy()
+    sub.w_idx = wl.w_idx
+    sub.planted = getattr(wl, "planted", None)
+    return sub
+
+
+def oracle_sample_time(wl, idxk_host, S: int):
+    """The oracle's layer group on the first S sequences of the workload, on
+    one host core: (seconds, S).  Main-KV codes are left zero: the oracle's
+    work (full scoring, full sorts, fp64 attention over every selected row)
+    does not depend on their values, and regenerating the selected rows of a
+    shuffled multi-GB page pool would dominate the sample."""
+    import oracle
+    sub = sub_workload(wl, S)
+    dm = oracle.dims()
+    kv = oracle.KV(np.zeros((wl.pool_rows, 256), np.uint8), np.zeros((wl.pool_rows, 32), np.uint8),
+                   idxk_host, seq_stride=wl.seq_stride, page_table=sub.page_table)
+    t0 = time.perf_counter()
+    oracle.layer_group(kv, dm, sub.n_rows, sub.modes, sub.q_idx, sub.w_h, sub.q, sub.swa,
+                       sub.swa_len, top_k=sub.top_k, pool_blocks=sub.pool_blocks)
+    return time.perf_counter() - t0, S
+
+
+def setup_device_workload(csa2, wl, dev):
+    """Device copies of a workload: its FP4 cache packed by the library's
+    pack kernel from the seeded bf16 rows, its indexer K and per-layer
+    inputs, a layer group and its workspace."""
+    import torch
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(dev)
+
+    rows = wl.pool_rows
+    codes = torch.empty((rows, 256), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, 32), dtype=torch.uint8, device=dev)
+    idxk = torch.empty((rows, 64), dtype=torch.int16, device=dev)
+    for r0, xc, kc in wl.iter_chunks():
+        n = len(xc)
+        csa2.csa2_quantize_fp4(to_dev(xc).view(torch.bfloat16), codes[r0:r0 + n],
+                               scales[r0:r0 + n])
+        idxk[r0:r0 + n] = to_dev(kc)
+    n_rows = to_dev(wl.n_rows.astype(np.int32))
+    pt = None if wl.page_table is None else to_dev(wl.page_table)
+    kv = csa2.KVCache(codes, scales, idxk, n_rows, max_rows=int(wl.n_rows.max()),
+                      seq_stride=wl.seq_stride, page_table=pt)
+    bufs = dict(q_idx=to_dev(wl.q_idx), w_h=to_dev(wl.w_h), q=to_dev(wl.q), swa=to_dev(wl.swa),
+                swa_len=to_dev(wl.swa_len))
+    grp = csa2.LayerGroup(kv, wl.modes, bufs["q_idx"], bufs["w_h"], bufs["q"], bufs["swa"],
+                          bufs["swa_len"], top_k=wl.top_k, pool_blocks=wl.pool_blocks)
+    ws = csa2.workspace(grp.workspace_size(), device=dev)
+    csa2.csa2_workspace_init(ws)
+    return dict(codes=codes, scales=scales, idxk=idxk, n_rows=n_rows, pt=pt, kv=kv, grp=grp,
+                ws=ws, **bufs)
+
+
+def units_of(wl) -> int:
+    return int(wl.B * wl.L)
+
+
+def time_back_to_back(csa2, wl, kv, bufs, ws, stream, K, W, copies: int = 3):
+    """Decode steps launched back to back, as a serving loop runs them, with
+    no L2 flush: the step's large inputs are kept out of L2 by rotating over
+    `copies` copies of the cache (each step streams its copy's indexer K,
+    larger than L2, and the copy it reads was last touched `copies` steps
+    earlier).  One event pair around all K steps.  Returns ms per step and
+    whether every copy's step reproduces the first copy's outputs."""
+    import torch
+    q_idx, w_h, q, swa, swa_len = bufs
+    groups, caches = [], []
+    for i in range(copies):
+        if i == 0:
+            kvi = kv
+        else:
+            c = (kv.codes.clone(), kv.scales.clone(), kv.idx_k.clone())
+            caches.append(c)
+            kvi = csa2.KVCache(c[0], c[1], c[2], kv.n_rows, max_rows=int(kv.view.max_rows),
+                               seq_stride=int(kv.view.seq_stride), page_table=kv.page_table)
+        groups.append(csa2.LayerGroup(kvi, wl.modes, q_idx, w_h, q, swa, swa_len,
+                                      top_k=wl.top_k, pool_blocks=wl.pool_blocks))
+    wss = [ws] + [csa2.workspace(groups[i].workspace_size(), device=q.device)
+                  for i in range(1, copies)]
+    for w_ in wss[1:]:
+        csa2.csa2_workspace_init(w_)
+    runs = []
+    for g, w_ in zip(groups, wss):
+        csa2.csa2_layer_group(g, w_)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            csa2.csa2_layer_group(g, w_)
+        runs.append(graph.replay)
+    for i in range(W * copies):
+        runs[i % copies]()
+    torch.cuda.synchronize()
+    same = all(torch.equal(g.idx, groups[0].idx) and torch.equal(g.out, groups[0].out)
+               for g in groups[1:])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        runs[i % copies]()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    for w_ in wss:
+        csa2.csa2_sync_status(w_)
+    ms = e0.elapsed_time(e1) / K
+    del runs, groups, caches
+    return ms, same
+
+
+def time_workload(csa2, k, dev, stream, flush_l2, K, W, with_cpu, cpu_seqs):
+    """A whole layer-group step of config k (the 8 x 131,072 HSI group or the
+    64 ragged paged sequences), timed like the headline step: one CUDA graph
+    per step, L2 flushed between steps, events around each step; a traced
+    pass gives the scan's own duration for its roofline; the oracle runs on
+    the first cpu_seqs sequences."""
+    import torch
+    from fp4_kv_cache_quantize_b200 import synth
+    wl = synth.config(k)
+    d = setup_device_workload(csa2, wl, dev)
+    grp, ws = d["grp"], d["ws"]
+    for _ in range(W):
+        csa2.csa2_layer_group(grp, ws)
+    torch.cuda.synchronize()
+    csa2.csa2_sync_status(ws)
+    launch = "direct"
+    run = lambda: csa2.csa2_layer_group(grp, ws)  # noqa: E731
+    try:
+        ref = grp.idx.clone()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            csa2.csa2_layer_group(grp, ws)
+        torch.cuda.synchronize()
+        grp.idx.fill_(-9)
+        graph.replay()
+        torch.cuda.synchronize()
+        if torch.equal(grp.idx, ref):
+            run, launch = graph.replay, "cuda_graph"
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        torch.cuda.synchronize()
+        launch = f"direct ({type(exc).__name__}: {exc})"[:200]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for i in range(K):
+        flush_l2()
+        ev[i][0].record(stream)
+        run()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    csa2.csa2_sync_status(ws)
+    times = sorted(a.elapsed_time(b) for a, b in ev)
+    ms = sum(times) / K
+    try:
+        bms, bsame = time_back_to_back(csa2, wl, d["kv"], (d["q_idx"], d["w_h"], d["q"], d["swa"],
+                                                          d["swa_len"]), ws, stream, K, W)
+        b2b = {"ms_per_step": bms, "value": units_of(wl) / (bms * 1e-3), "copies_agree": bool(bsame)}
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        b2b = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        torch.cuda.synchronize()
+    # traced pass: the scan's duration
+    n_ev, KT = 32, min(K, 10)
+    tev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev * KT)]
+    for e in tev:
+        e.record(stream)
+    torch.cuda.synchronize()
+    scan_ms, stages = [], {}
+    for i in range(KT):
+        tr = csa2.Trace(tev[i * n_ev:(i + 1) * n_ev])
+        flush_l2()
+        csa2.csa2_trace_set(tr)
+        csa2.csa2_layer_group(grp, ws)
+        csa2.csa2_trace_set(None)
+        torch.cuda.synchronize()
+        names = tr.names()
+        for j in range(len(names) - 1):
+            dt = tr.events[j].elapsed_time(tr.events[j + 1])
+            stages[names[j]] = stages.get(names[j], 0.0) + dt * 1e3 / KT
+            if names[j] == "scan":
+                scan_ms.append(dt)
+    ab = algorithmic_bytes(wl)
+    peak, peak_kind = measured_peaks()
+    units = wl.B * wl.L
+    out = {"workload": wl.name, "value": units / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+           "steps": K, "warmup": W, "step_launch": launch,
+           "step_ms_p10_p50_p90": [float(np.percentile(times, p)) for p in (10, 50, 90)],
+           "algorithmic_bytes_per_step": ab["total"],
+           "hbm_gbs_algorithmic": ab["total"] / (ms * 1e-3) / 1e9,
+           "frac_of_measured_hbm": ab["total"] / (ms * 1e-3) / 1e9 / peak,
+           "stage_us": stages, "back_to_back": b2b, "config": config_dict(wl)}
+    if scan_ms:
+        t_scan = sum(scan_ms) / len(scan_ms) * 1e-3
+        out["roofline"] = {"bound": "hbm", "kernel": "score_scan_kernel",
+                           "achieved": ab["scan"] / t_scan / 1e9, "peak": peak,
+                           "peak_kind": peak_kind, "unit": "GB/s",
+                           "frac": ab["scan"] / t_scan / 1e9 / peak, "traffic": None,
+                           "algorithmic_bytes_per_launch": ab["scan"]}
+    if with_cpu:
+        S = min(cpu_seqs, wl.B)
+        idxk_host = d["idxk"].cpu().numpy().view(np.uint16)
+        dt, S = oracle_sample_time(wl, idxk_host, S)
+        out["cpu_baseline"] = {"value": S * wl.L / dt, "unit": UNIT, "cores": 1,
+                               "kind": "oracle",
+                               "sample": (f"one step of the first {S} of the {wl.B} sequences "
+                                          f"of {wl.name} on one host core (fp64 C oracle; "
+                                          "main-KV codes zero, the oracle's work does not "
+                                          "depend on them)")}
+    del d, grp, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_quant(csa2, dev, stream, K, W, with_cpu):
+    """The FP4 quantise / dequantise microbenchmark: 1,048,576 x 512 bf16
+    rows (0.1% of elements x50) packed to E2M1 codes and E4M3 scales by one
+    launch, and unpacked again by one launch.  The 1 GiB input exceeds L2,
+    so calls run back to back between two events."""
+    import torch
+    from fp4_kv_cache_quantize_b200 import synth
+    wl = synth.config(1)
+    rows = wl.pool_rows
+    x = torch.empty((rows, 512), dtype=torch.int16, device=dev)
+    for c in range(wl.n_chunks):
+        xc = wl.x_chunk(c)
+        r0 = c * synth.CHUNK_ROWS
+        x[r0:r0 + len(xc)] = torch.from_numpy(xc.view(np.int16)).to(dev)
+    xb = x.view(torch.bfloat16)
+    codes = torch.empty((rows, 256), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, 32), dtype=torch.uint8, device=dev)
+    y = torch.empty((rows, 512), dtype=torch.bfloat16, device=dev)
+    nbytes = rows * QUANT_BYTES_PER_ROW
+    peak, peak_kind = measured_peaks()
+    out = {"workload": wl.name, "rows": rows, "channels": 512,
+           "algorithmic_bytes_per_launch": nbytes}
+    for name, fn in (("quantize", lambda: csa2.csa2_quantize_fp4(xb, codes, scales)),
+                     ("dequantize", lambda: csa2.csa2_dequantize_fp4(codes, scales, y))):
+        for _ in range(W):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / K * 1e-3
+        gbs = nbytes / t / 1e9
+        out[name] = {"us_per_launch": t * 1e6, "value": gbs, "unit": "GB/s",
+                     "roofline": {"bound": "hbm", "kernel": f"fp4_{'pack' if name == 'quantize' else 'unpack'}_kernel",
+                                  "achieved": gbs, "peak": peak, "peak_kind": peak_kind,
+                                  "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+                     "timing": f"{K} back-to-back launches after {W}, CUDA events (1 GiB input > L2)"}
+    if with_cpu:
+        import oracle
+        S = 16384
+        xs = wl.x_chunk(0)
+        for c in range(1, S // synth.CHUNK_ROWS):
+            xs = np.concatenate([xs, wl.x_chunk(c)])
+        t0 = time.perf_counter()
+        oracle.quantize_fp4(xs)
+        dt = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": S * QUANT_BYTES_PER_ROW / dt / 1e9, "unit": "GB/s",
+                               "cores": 1, "kind": "oracle",
+                               "sample": f"the oracle's quantiser on the first {S} rows"}
+    del x, codes, scales, y
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, wl, rank, world):
     import torch
 
@@ -676,6 +956,22 @@ def run_gpu(args, wl, rank, world):
     csa2.csa2_sync_status(ws)
     times = [a.elapsed_time(b) for a, b in ev]   # ms
     t_step = max_over_ranks(sum(times) / K, dist, dev)
+
+    # ---- the same steps back to back (no flush; the cache rotates over three
+    # copies so that every step's large inputs are cold in L2)
+    try:
+        b2b_ms, b2b_same = time_back_to_back(csa2, wl, kv, (q_idx, w_h, q, swa, swa_len), ws,
+                                             stream, K, args.warmup)
+        b2b_ms = max_over_ranks(b2b_ms, dist, dev)
+        b2b = {"ms_per_step": b2b_ms, "value": job_throughput(wl.B * wl.L, world, b2b_ms),
+               "unit": UNIT, "copies_agree": bool(b2b_same),
+               "timing": (f"{K} steps back to back between two events after warm-up, no L2 "
+                          "flush: the steps rotate over three copies of the cache, so every "
+                          "step streams indexer K that the two steps before it did not touch "
+                          "(3 x 134 MB > the 126 MB L2)")}
+    except Exception as exc:  # noqa: BLE001  (reported in the line)
+        b2b = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        torch.cuda.synchronize()
 
     # ---- traced pass: per-launch events for the stage breakdown and roofline
     n_ev = 32
@@ -795,6 +1091,20 @@ def run_gpu(args, wl, rank, world):
         cpar = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         quiet_sync()
 
+    others = {}
+    for key_, fn in (("fp4_quant_1Mx512", lambda: time_quant(csa2, dev, stream, 20, 3, with_cpu)),
+                     ("hsi_group_b8_128k", lambda: time_workload(csa2, 2, dev, stream, flush_l2,
+                                                                 max(10, K // 2), 3, with_cpu, 8)),
+                     ("ragged_paged_64seq_r2", lambda: time_workload(
+                         csa2, 4, dev, stream, flush_l2, max(10, K // 2), 3, with_cpu, 4))):
+        if args.skip_configs:
+            break
+        try:
+            others[key_] = fn()
+        except Exception as exc:  # noqa: BLE001  (reported in the line)
+            others[key_] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            quiet_sync()
+
     units = wl.B * wl.L
     value = job_throughput(units, world, t_step)
     ab = algorithmic_bytes(wl)
@@ -830,6 +1140,8 @@ def run_gpu(args, wl, rank, world):
                                "output, indices) copied back, on separate streams overlapping "
                                "the neighbouring steps' compute; no L2 flush (134 MB of "
                                "indexer K per step exceeds the 126 MB L2)")},
+            "back_to_back": b2b,
+            "configs": others,
             "layer_sequential": seq,
             "next_rows": {"cache_append": append, "multi_query": multi,
                           "prefill_chunk": prefill, "context_parallel": cpar},
@@ -851,6 +1163,8 @@ def main():
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--skip-configs", action="store_true",
+                    help="time only the headline workload (not configs 1, 2 and 4)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", 0))

@@ -60,20 +60,20 @@ constexpr uint32_t TA_O_COL = 64;
 
 struct TaSmem {
   // K = V in fp16: channel block kb at kb * TA_KB, 128 rows (keys) of 128 B,
-  // 16-byte chunks swizzled by row % 8
+  // 16-byte chunks swizzled by row % 8.  Before the rows are dequantised it
+  // holds the raw bf16 queries.
   alignas(1024) uint8_t tile[8 * TA_KB];
   alignas(1024) uint8_t q[8 * 2048];       // Q': channel block kb, 16 rows (heads) of 128 B
   alignas(1024) uint8_t p[2 * 2048];       // P^T: key block kb, 16 rows (heads) of 128 B
   // gathered rows: the window's E4M3 rows, or FP4 codes | scales | the
-  // normalised partials this CTA receives as the owner of a channel block
+  // normalised partials this CTA receives as the owner of a channel block;
+  // after the dequantisation its first 8 KB hold the logits [head][key]
   alignas(16) uint8_t raw[TA_RAW_BYTES];
   int64_t row[TA_KEYS];
   float scl1[CSA2_H], scl2[CSA2_H];        // logit = acc * scl1 * scl2 (log2 units)
-  uint32_t qmax[TA_NT / 32][4];
-  float wmax[4][CSA2_H];
-  float m[CSA2_H], lsum[CSA2_H];
+  float m[CSA2_H], lsum[CSA2_H], linv[CSA2_H];
   float2 ml[TA_CTAS][CSA2_H];              // (max, sum) per source CTA, at the owners
-  float wts[TA_CTAS][CSA2_H];
+  alignas(16) float wts[TA_CTAS][CSA2_H];
   uint64_t mbar;
   uint32_t tmem_base;
 };
@@ -101,6 +101,9 @@ __device__ __forceinline__ uint32_t sw_off(int r, int cc) {
   return (uint32_t)(r * 128 + ((cc ^ (r & 7)) << 4));
 }
 
+// The code below runs once per CTA: every instruction is fetched cold, so
+// loops are kept rolled (a rolled loop body is fetched once, an unrolled one
+// costs its full length in instruction fetch).
 __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   TaSmem& s = *reinterpret_cast<TaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -121,54 +124,13 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     tmem_alloc(&s.tmem_base, TA_TMEM_COLS);
     tmem_relinquish();
   }
-
-  // ---- Q' = Q * 2^e_h in fp16: max |Q'_h| in [2^14, 2^15).  The queries
-  // are inputs (no kernel of this library writes them): read before the wait.
-  uint4 qv[4];
+  // The queries are inputs (no kernel of this library writes them): their
+  // copy into shared memory starts before the wait for the indices.
   {
-    const uint4* qg = reinterpret_cast<const uint4*>(L.q + (int64_t)b * CSA2_H * CSA2_D);
-#pragma unroll
-    for (int u = 0; u < 4; u++) {  // chunk t + 256 u: head (t >> 6) + 4 u, chunk t & 63
-      qv[u] = __ldg(qg + t + TA_NT * u);
-      const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
-      uint32_t mx = 0u;
-#pragma unroll
-      for (int k = 0; k < 4; k++) mx = max(mx, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
-      mx = __reduce_max_sync(0xffffffffu, mx);
-      if (lane == 0) s.qmax[warp][u] = mx;
-    }
-  }
-  __syncthreads();
-  {
-    const int hq = t >> 6, cfull = t & 63, kb = cfull >> 3, cc = cfull & 7;
-#pragma unroll
-    for (int u = 0; u < 4; u++) {
-      const int h = hq + 4 * u;
-      const uint32_t mb = max(s.qmax[warp][u], s.qmax[warp ^ 1][u]);
-      const float M = __uint_as_float(mb << 16);
-      int e = 0;
-      if (M > 0.0f && M <= 3.3895314e38f) {  // finite, nonzero: 2^14 <= M 2^e < 2^15
-        int ex;
-        frexpf(M, &ex);
-        e = 15 - ex;
-      }
-      const int e1 = e / 2, e2 = e - e1;  // each within a float's exponent range
-      const float f1 = pow2i(e1), f2 = pow2i(e2);
-      if (cfull == 0) {
-        s.scl1[h] = pow2i(-e1);
-        s.scl2[h] = p.scale_log2 * pow2i(-e2);
-      }
-      const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
-      uint32_t o4[4];
-#pragma unroll
-      for (int k = 0; k < 4; k++) {
-        const float lo = __uint_as_float(w[k] << 16) * f1 * f2;
-        const float hi = __uint_as_float(w[k] & 0xFFFF0000u) * f1 * f2;
-        o4[k] = h2u(__floats2half2_rn(lo, hi));
-      }
-      *reinterpret_cast<uint4*>(s.q + kb * 2048 + sw_off(h, cc)) =
-          make_uint4(o4[0], o4[1], o4[2], o4[3]);
-    }
+    const uint8_t* qg = reinterpret_cast<const uint8_t*>(L.q + (int64_t)b * CSA2_H * CSA2_D);
+#pragma unroll 1
+    for (int i = t; i < CSA2_H * CSA2_D * 2 / 16; i += TA_NT) cp_async16(s.tile + 16 * i, qg + 16 * i);
+    cp_async_commit();
   }
   tc_fence_before();
   __syncthreads();
@@ -181,6 +143,11 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   // sequence bp sees the sequence's entries minus the drafts after it, and
   // the window rows that end at its own entry.
   const int bp = b / p.nq, tq = b - bp * p.nq, later = p.nq - 1 - tq;
+  // this thread's index, read before the counts arrive (within the index
+  // array's stride either way): the three loads are in flight together
+  const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
+  const int kt = c * TA_KEYS + t;
+  const int pos_t = !window && t < TA_KEYS && kt < p.idx_stride ? __ldg(idx + kt) : -1;
   int C = p.n_rows[bp];
   if (C < 0 || C > p.max_rows) {
     if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
@@ -188,6 +155,7 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   }
   C = C - later < 0 ? 0 : C - later;
   int nk;  // candidate keys of this CTA: keys j < nk
+  const uint8_t* wbase = nullptr;
   if (!window) {
     int n_idx = L.idx_count[b];
     if (n_idx < 0 || n_idx > p.idx_stride) {
@@ -196,17 +164,14 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     }
     const int k0 = c * TA_KEYS;
     nk = min(max(n_idx - k0, 0), TA_KEYS);
-    const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
     if (L.idx_copy) {  // Reuse layer: publish the indices it used
-      for (int i = t; i < TA_KEYS && k0 + i < p.idx_stride; i += TA_NT)
-        L.idx_copy[(int64_t)b * p.idx_stride + k0 + i] = idx[k0 + i];
+      if (t < TA_KEYS && kt < p.idx_stride) L.idx_copy[(int64_t)b * p.idx_stride + kt] = pos_t;
       if (c == 0 && t == 0) L.idx_copy_count[b] = L.idx_count[b];
     }
     if (t < TA_KEYS) {
       int64_t row = -1;
       if (t < nk) {
-        const int pos = __ldg(idx + k0 + t);
-        if (pos >= 0 && pos < C) row = ta_kv_row(p, bp, pos);
+        if (pos_t >= 0 && pos_t < C) row = ta_kv_row(p, bp, pos_t);
         if (row < 0) set_status(p.status, ST_DEVICE_CHECK);
       }
       s.row[t] = row;
@@ -220,66 +185,105 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     const int win_end = n_win - later < 0 ? 0 : n_win - later;
     const int win_lo = win_end > CSA2_W ? win_end - CSA2_W : 0;
     nk = win_end - win_lo;
-    if (t < TA_KEYS) s.row[t] = t < nk ? (int64_t)(win_lo + t) : -1;
+    wbase = L.swa + ((int64_t)bp * p.swa_rows + win_lo) * CSA2_D;
+    if (t < TA_KEYS) s.row[t] = t < nk ? (int64_t)t : -1;
   }
   __syncthreads();
 
   // ---- gather the rows (16-byte asynchronous copies)
   if (nk > 0) {
     if (!window) {
-#pragma unroll
-      for (int u = 0; u < (TA_KEYS * 18 + TA_NT - 1) / TA_NT; u++) {
-        const int i = t + TA_NT * u;
+#pragma unroll 1
+      for (int i = t; i < TA_KEYS * 18; i += TA_NT) {
         const int r = i / 18, part = i - 18 * r;
-        if (r < TA_KEYS) {
-          const int64_t row = s.row[r];
-          if (row >= 0) {
-            if (part < 16)
-              cp_async16(s.raw + r * TA_CODE_LD + 16 * part, p.codes + row * (CSA2_D / 2) + 16 * part);
-            else
-              cp_async16(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * (part - 16),
-                         p.scales + row * (CSA2_D / 16) + 16 * (part - 16));
-          }
+        const int64_t row = s.row[r];
+        if (row >= 0) {
+          if (part < 16)
+            cp_async16(s.raw + r * TA_CODE_LD + 16 * part, p.codes + row * (CSA2_D / 2) + 16 * part);
+          else
+            cp_async16(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * (part - 16),
+                       p.scales + row * (CSA2_D / 16) + 16 * (part - 16));
         }
       }
     } else {
-      const uint8_t* swa = L.swa + (int64_t)bp * p.swa_rows * CSA2_D;
-#pragma unroll 4
-      for (int u = 0; u < TA_KEYS * 32 / TA_NT; u++) {
-        const int i = t + TA_NT * u, r = i >> 5, part = i & 31;
-        const int64_t row = s.row[r];
-        if (row >= 0) cp_async16(s.raw + r * TA_WIN_LD + 16 * part, swa + row * CSA2_D + 16 * part);
+#pragma unroll 1
+      for (int i = t; i < TA_KEYS * 32; i += TA_NT) {
+        const int r = i >> 5, part = i & 31;
+        if (s.row[r] >= 0) cp_async16(s.raw + r * TA_WIN_LD + 16 * part, wbase + r * CSA2_D + 16 * part);
       }
     }
-    cp_async_commit();
-    cp_async_wait_all();
   }
+  cp_async_commit();  // the rows' group (empty when there are none)
+  // the queries' copies (the first group) have landed; the rows may still be
+  // in flight while the queries are converted
+  asm volatile("cp.async.wait_group %0;" ::"n"(1) : "memory");
   __syncthreads();
+
+  // ---- Q' = Q * 2^e_h in fp16, max |Q'_h| in [2^14, 2^15): 16 threads per
+  // head, 32 channels each
+  {
+    const int h = t >> 4, g = t & 15;
+    const uint4* src = reinterpret_cast<const uint4*>(s.tile + h * (CSA2_D * 2) + g * 64);
+    uint4 v[4];
+    uint32_t mx = 0u;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      v[k] = src[k];
+      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; j++) mx = max(mx, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float M = __uint_as_float(mx << 16);
+    int e = 0;
+    if (M > 0.0f && M <= 3.3895314e38f) {  // finite, nonzero: 2^14 <= M 2^e < 2^15
+      int ex;
+      frexpf(M, &ex);
+      e = 15 - ex;
+    }
+    const int e1 = e / 2, e2 = e - e1;  // each within a float's exponent range
+    const float f = pow2i(e1), f2 = pow2i(e2);
+    if (g == 0) {
+      s.scl1[h] = pow2i(-e1);
+      s.scl2[h] = p.scale_log2 * pow2i(-e2);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; k++) {  // channels 32 g + 8 k .. + 8: block g / 2, chunk 4 (g & 1) + k
+      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int j = 0; j < 4; j++)
+        o4[j] = h2u(__floats2half2_rn(__uint_as_float(w[j] << 16) * f * f2,
+                                      __uint_as_float(w[j] & 0xFFFF0000u) * f * f2));
+      *reinterpret_cast<uint4*>(s.q + (g >> 1) * 2048 + sw_off(h, 4 * (g & 1) + k)) =
+          make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();  // the rows have landed; the raw queries in the tile are consumed
 
   // ---- dequantise into the fp16 tile: two threads per row, 256 channels each
   if (nk > 0) {
     const int r = t & (TA_KEYS - 1), half = t >> 7;
-    const bool valid = s.row[r] >= 0;
-    uint8_t* trow = s.tile;
-    if (!valid) {
-#pragma unroll
-      for (int j = 0; j < 32; j++) {
-        const int kb = 4 * half + (j >> 3), cc = j & 7;
-        *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc)) = make_uint4(0, 0, 0, 0);
-      }
+    uint8_t* trow = s.tile + r * 128;
+    const int sw = r & 7;
+    if (s.row[r] < 0) {
+#pragma unroll 1
+      for (int j = 0; j < 32; j++)
+        *reinterpret_cast<uint4*>(trow + (4 * half + (j >> 3)) * TA_KB + (((j & 7) ^ sw) << 4)) =
+            make_uint4(0, 0, 0, 0);
     } else if (!window) {
       const uint8_t* cr = s.raw + r * TA_CODE_LD + 128 * half;
-      const uint4 sc = *reinterpret_cast<const uint4*>(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD +
-                                                       16 * half);
-      const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
-#pragma unroll
+      const uint8_t* sr = s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * half;
+#pragma unroll 1
       for (int i = 0; i < 8; i++) {  // 16 code bytes: channels 256 half + 32 i + [0, 32)
         const uint4 cv = *reinterpret_cast<const uint4*>(cr + 16 * i);
         const uint32_t words[4] = {cv.x, cv.y, cv.z, cv.w};
-        const uint32_t sb = (scw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;  // groups 2i, 2i+1
+        const uint32_t sb = *reinterpret_cast<const uint16_t*>(sr + 2 * i);  // groups 2i, 2i+1
         const __half s0 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sb & 0xFF), __NV_E4M3));
         const __half s1 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sb >> 8), __NV_E4M3));
-        const int kb = 4 * half + (i >> 1);
+        uint8_t* dst = trow + (4 * half + (i >> 1)) * TA_KB;
 #pragma unroll
         for (int q4 = 0; q4 < 4; q4++) {  // 8 channels per 16-byte store
           const uint32_t word = words[q4];
@@ -290,14 +294,13 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
             hv[k] = h2u(__hmul2(__half2(__nv_cvt_fp4x2_to_halfraw2(
                                     (__nv_fp4x2_storage_t)((word >> (8 * k)) & 0xFF), __NV_E2M1)),
                                 scv));
-          const int cc = 4 * (i & 1) + q4;
-          *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc)) =
+          *reinterpret_cast<uint4*>(dst + (((4 * (i & 1) + q4) ^ sw) << 4)) =
               make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
       }
     } else {
       const uint8_t* wr = s.raw + r * TA_WIN_LD + 256 * half;
-#pragma unroll
+#pragma unroll 1
       for (int j = 0; j < 16; j++) {  // 16 E4M3 bytes: channels 256 half + 16 j + [0, 16)
         const uint4 v = *reinterpret_cast<const uint4*>(wr + 16 * j);
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -309,11 +312,10 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
           hv[2 * k + 1] = h2u(__half2(__nv_cvt_fp8x2_to_halfraw2(
               (__nv_fp8x2_storage_t)(wv[k] >> 16), __NV_E4M3)));
         }
-        const int kb = 4 * half + (j >> 2), cc = 2 * (j & 3);
-        *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc)) =
-            make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        *reinterpret_cast<uint4*>(trow + kb * TA_KB + sw_off(r, cc + 1)) =
-            make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        uint8_t* dst = trow + (4 * half + (j >> 2)) * TA_KB;
+        const int cc = 2 * (j & 3);
+        *reinterpret_cast<uint4*>(dst + ((cc ^ sw) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ sw) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
       }
     }
     fence_proxy_async_smem();
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   if (nk > 0 && t == 0) {
     tc_fence_after();
     const uint32_t a0 = smem_u32(s.tile), b0 = smem_u32(s.q);
-#pragma unroll
+#pragma unroll 1
     for (int kb = 0; kb < 8; kb++)
 #pragma unroll
       for (int sub = 0; sub < 4; sub++)
@@ -333,9 +335,9 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
                   TA_IDESC_QK, (kb | sub) != 0);
     umma_commit(&s.mbar);
   }
+  float* sS = reinterpret_cast<float*>(s.raw);  // logits [head][key], log2 units
   bool ok = true;
   if (nk > 0 && warp < 4) {
-    // ---- softmax over this CTA's keys: thread = key, 16 heads
     ok = __all_sync(0xffffffffu, mbar_wait(&s.mbar, 0, nullptr));
     if (!ok && lane == 0) set_status(p.status, ST_TIMEOUT);
     tc_fence_after();
@@ -344,23 +346,46 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     tmem_ld_wait();
     const int key = 32 * warp + lane;
     const bool valid = ok && key < nk && s.row[key] >= 0;
-    float x[16];
 #pragma unroll
-    for (int h = 0; h < 16; h++) {
-      x[h] = valid ? __uint_as_float(r[h]) * s.scl1[h] * s.scl2[h] : -INFINITY;
-      const float mh = warp_max_f32(x[h]);
-      if (lane == h) s.wmax[warp][h] = mh;
+    for (int h = 0; h < 16; h++)
+      sS[h * TA_KEYS + key] = valid ? __uint_as_float(r[h]) * s.scl1[h] * s.scl2[h] : -INFINITY;
+  }
+  __syncthreads();
+  // ---- softmax: 16 threads per head, 8 keys each; P^T in fp16, the sum
+  // of the fp16 probabilities the MMA reads
+  if (nk > 0) {
+    const int h = t >> 4, g = t & 15;
+    const float4* src = reinterpret_cast<const float4*>(sS + h * TA_KEYS + 8 * g);
+    const float4 x0 = src[0], x1 = src[1];
+    float m = fmaxf(fmaxf(fmaxf(x0.x, x0.y), fmaxf(x0.z, x0.w)),
+                    fmaxf(fmaxf(x1.x, x1.y), fmaxf(x1.z, x1.w)));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint32_t pv[4];
+    float l = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const __half2 ph = m == -INFINITY ? __floats2half2_rn(0.0f, 0.0f)
+                                        : __floats2half2_rn(exp2f(xs[2 * k] - m),
+                                                            exp2f(xs[2 * k + 1] - m));
+      const float2 pf = __half22float2(ph);
+      l += pf.x + pf.y;
+      pv[k] = h2u(ph);
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const int kb = key >> 6, cc = (key & 63) >> 3;
+    *reinterpret_cast<uint4*>(s.p + (g >> 3) * 2048 + sw_off(h, g & 7)) =
+        make_uint4(pv[0], pv[1], pv[2], pv[3]);
 #pragma unroll
-    for (int h = 0; h < 16; h++) {
-      const float m = fmaxf(fmaxf(s.wmax[0][h], s.wmax[1][h]), fmaxf(s.wmax[2][h], s.wmax[3][h]));
-      const float pe = m == -INFINITY ? 0.0f : exp2f(x[h] - m);
-      *reinterpret_cast<__half*>(s.p + kb * 2048 + sw_off(h, cc) + (key & 7) * 2) = __float2half_rn(pe);
-      if (lane == h && warp == 0) s.m[h] = m;
+    for (int o = 8; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (g == 0) {
+      s.m[h] = m;
+      s.lsum[h] = l;
+      s.linv[h] = l > 0.0f ? 1.0f / l : 0.0f;
     }
     fence_proxy_async_smem();
+  } else if (t < CSA2_H) {
+    s.m[t] = -INFINITY;
+    s.lsum[t] = 0.0f;
   }
   tc_fence_before();
   __syncthreads();
@@ -369,78 +394,46 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   if (nk > 0 && t == 0) {
     tc_fence_after();
     const uint32_t a0 = smem_u32(s.tile), b0 = smem_u32(s.p);
-#pragma unroll
-    for (int cb = 0; cb < 4; cb++)
-#pragma unroll
-      for (int ks = 0; ks < 8; ks++)
-        umma_bf16(tmem + TA_O_COL + 16 * cb,
-                  sdesc_mn128(a0 + cb * 2 * TA_KB + ks * 2048, TA_KB, 1024),
-                  sdesc_k128(b0 + (ks >> 2) * 2048 + (ks & 3) * 32), TA_IDESC_PV, ks > 0);
+#pragma unroll 1
+    for (int i = 0; i < 32; i++) {
+      const int cb = i >> 3, ks = i & 7;
+      umma_bf16(tmem + TA_O_COL + 16 * cb, sdesc_mn128(a0 + cb * 2 * TA_KB + ks * 2048, TA_KB, 1024),
+                sdesc_k128(b0 + (ks >> 2) * 2048 + (ks & 3) * 32), TA_IDESC_PV, ks > 0);
+    }
     umma_commit(&s.mbar);
   }
-  if (warp >= 4) {
-    // ---- the softmax sums from the fp16 probabilities the MMA reads:
-    // 8 threads per head, 16 keys each
-    const int u = t - 128, h = u >> 3, seg = u & 7;
-    float l = 0.0f;
-    if (nk > 0) {
-#pragma unroll
-      for (int k2 = 0; k2 < 2; k2++) {
-        const int cc = 2 * (seg & 3) + k2;
-        const uint4 v = *reinterpret_cast<const uint4*>(s.p + (seg >> 2) * 2048 + sw_off(h, cc));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          l += f.x + f.y;
-        }
-      }
-    }
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    if (seg == 0) s.lsum[h] = l;
-  }
-  if (nk == 0 && t < CSA2_H) s.m[t] = -INFINITY;
-  __syncthreads();
 
-  // ---- normalised partial O^T -> the owners of the channel blocks
-  if (warp < 4) {
-    uint32_t o[4][16];
-    bool ok2 = ok;
-    if (nk > 0) {
-      ok2 = __all_sync(0xffffffffu, ok && mbar_wait(&s.mbar, 1, nullptr));
-      if (!ok2 && lane == 0 && ok) set_status(p.status, ST_TIMEOUT);
-      tc_fence_after();
-#pragma unroll
-      for (int cb = 0; cb < 4; cb++)
-        tmem_ld_x16(tmem + ((uint32_t)(32 * warp) << 16) + TA_O_COL + 16 * cb, o[cb]);
+  // ---- normalised partial O^T -> the owners of the channel blocks: warp w
+  // reads TMEM lanes 32 (w % 4).., channel blocks 2 (w / 4) and 2 (w / 4) + 1
+  bool live = nk > 0 && ok;
+  if (nk > 0) {
+    const bool done = __all_sync(0xffffffffu, ok && mbar_wait(&s.mbar, 1, nullptr));
+    if (!done && ok && lane == 0) set_status(p.status, ST_TIMEOUT);
+    live = __syncthreads_and(done);
+  }
+  if (live) {
+    tc_fence_after();
+    const int chl = 32 * (warp & 3) + lane;
+#pragma unroll 1
+    for (int cb = 2 * (warp >> 2); cb < 2 * (warp >> 2) + 2; cb++) {
+      uint32_t o[16];
+      tmem_ld_x16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + TA_O_COL + 16 * cb, o);
       tmem_ld_wait();
+      uint32_t hv[8];
+#pragma unroll
+      for (int k = 0; k < 8; k++)
+        hv[k] = h2u(__floats2half2_rn(__uint_as_float(o[2 * k]) * s.linv[2 * k],
+                                      __uint_as_float(o[2 * k + 1]) * s.linv[2 * k + 1]));
+      uint4* dst = reinterpret_cast<uint4*>(
+          cluster.map_shared_rank(s.raw + TA_RECV_OFF + ((c * 128 + chl) * CSA2_H) * 2, cb));
+      dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
     }
-    const bool live = nk > 0 && ok2;
-    if (live) {
-      float inv[16];
-#pragma unroll
-      for (int h = 0; h < 16; h++) inv[h] = s.lsum[h] > 0.0f ? 1.0f / s.lsum[h] : 0.0f;
-      const int chl = 32 * warp + lane;
-#pragma unroll
-      for (int cb = 0; cb < TA_SPARSE; cb++) {
-        uint32_t hv[8];
-#pragma unroll
-        for (int k = 0; k < 8; k++)
-          hv[k] = h2u(__floats2half2_rn(__uint_as_float(o[cb][2 * k]) * inv[2 * k],
-                                        __uint_as_float(o[cb][2 * k + 1]) * inv[2 * k + 1]));
-        uint4* dst = reinterpret_cast<uint4*>(cluster.map_shared_rank(
-            s.raw + TA_RECV_OFF + ((c * 128 + chl) * CSA2_H) * 2, cb));
-        dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-      }
-    }
-    if (t < CSA2_H) {
-      const float2 ml = live ? make_float2(s.m[t], s.lsum[t]) : make_float2(-INFINITY, 0.0f);
-#pragma unroll
-      for (int o2 = 0; o2 < TA_SPARSE; o2++) *cluster.map_shared_rank(&s.ml[c][t], o2) = ml;
-    }
+  }
+  if (t < CSA2_H) {
+    const float2 ml = live ? make_float2(s.m[t], s.lsum[t]) : make_float2(-INFINITY, 0.0f);
+#pragma unroll 1
+    for (int o2 = 0; o2 < TA_SPARSE; o2++) *cluster.map_shared_rank(&s.ml[c][t], o2) = ml;
   }
   tc_fence_before();
   __syncthreads();
@@ -468,30 +461,34 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
       for (int src = 0; src < TA_CTAS; src++) s.wts[src][t] = wv[src] * inv;
     }
     __syncthreads();
-    if (t < 128) {
-      float acc[16];
+    // two threads per channel, eight heads each
+    const int ch = t & 127, hh = 8 * (t >> 7);
+    float acc[8];
 #pragma unroll
-      for (int h = 0; h < 16; h++) acc[h] = 0.0f;
+    for (int k = 0; k < 8; k++) acc[k] = 0.0f;
+#pragma unroll 1
+    for (int src = 0; src < TA_CTAS; src++) {
+      const float4 w0 = *reinterpret_cast<const float4*>(&s.wts[src][hh]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&s.wts[src][hh + 4]);
+      if (w0.x == 0.0f && w0.y == 0.0f && w0.z == 0.0f && w0.w == 0.0f && w1.x == 0.0f &&
+          w1.y == 0.0f && w1.z == 0.0f && w1.w == 0.0f)
+        continue;  // nothing from this source for these heads (its buffer may be stale)
+      const uint4 v = *reinterpret_cast<const uint4*>(s.raw + TA_RECV_OFF +
+                                                      ((src * 128 + ch) * CSA2_H + hh) * 2);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      const float wt[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int src = 0; src < TA_CTAS; src++) {
-        const uint4* v =
-            reinterpret_cast<const uint4*>(s.raw + TA_RECV_OFF + ((src * 128 + t) * CSA2_H) * 2);
-        const uint4 v0 = v[0], v1 = v[1];
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int k = 0; k < 8; k++) {
-          const float wa = s.wts[src][2 * k], wb = s.wts[src][2 * k + 1];
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          if (wa != 0.0f) acc[2 * k] = fmaf(wa, f.x, acc[2 * k]);
-          if (wb != 0.0f) acc[2 * k + 1] = fmaf(wb, f.y, acc[2 * k + 1]);
-        }
+      for (int k = 0; k < 4; k++) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        acc[2 * k] = fmaf(wt[2 * k], f.x, acc[2 * k]);
+        acc[2 * k + 1] = fmaf(wt[2 * k + 1], f.y, acc[2 * k + 1]);
       }
-      uint16_t* out = L.out + (int64_t)b * CSA2_H * CSA2_D + c * 128 + t;
+    }
+    uint16_t* out = L.out + ((int64_t)b * CSA2_H + hh) * CSA2_D + c * 128 + ch;
 #pragma unroll
-      for (int h = 0; h < 16; h++) {
-        const __nv_bfloat16 v = __float2bfloat16_rn(acc[h]);
-        out[h * CSA2_D] = *reinterpret_cast<const uint16_t*>(&v);
-      }
+    for (int k = 0; k < 8; k++) {
+      const __nv_bfloat16 v = __float2bfloat16_rn(acc[k]);
+      out[k * CSA2_D] = *reinterpret_cast<const uint16_t*>(&v);
     }
   }
 }

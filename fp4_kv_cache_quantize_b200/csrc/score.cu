@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
     if (lane == 0) {  // ---------------------------------- TMA producer
       int stage = 0, cur_b = -1, C = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
+      const uint64_t stream_once = l2_policy_evict_first();  // indexer K is read once per step
       for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
         const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
         if (b != cur_b) {
@@ -165,8 +166,8 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
         const int32_t y0 = box_row(p, b, pos0);
         const int32_t y1 = pos0 + SC_BOX < C - p.tail ? box_row(p, b, pos0 + SC_BOX) : y0;
         mbar_arrive_expect_tx(&s.full[stage], SC_A_BYTES + Cfg::B_BYTES);
-        tma_load_2d(s.a[stage], &map_k, &s.full[stage], 0, y0);
-        tma_load_2d(s.a[stage] + SC_BOX * 128, &map_k, &s.full[stage], 0, y1);
+        tma_load_2d_hint(s.a[stage], &map_k, &s.full[stage], 0, y0, stream_once);
+        tma_load_2d_hint(s.a[stage] + SC_BOX * 128, &map_k, &s.full[stage], 0, y1, stream_once);
         tma_load_2d(s.b[stage], &map_q, &s.full[stage], 0, (b * p.nq + p.q_first) * CSA2_HI);
         issued |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -375,6 +376,12 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
   const int b = blockIdx.y;
   const RescoreJob job = p.job[blockIdx.z];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int e0 = rank * EPC;  // first candidate of this CTA
+  // the candidate blocks are read without waiting for their count (within
+  // the list's stride), so both loads are in flight together
+  int cblk = -1;
+  if (t < EPC / CSA2_BLK && e0 / CSA2_BLK + t < p.cand_stride)
+    cblk = p.cand[(int64_t)b * p.cand_stride + e0 / CSA2_BLK + t];
   const int C = visible_query(p.n_rows, b, p.nq, p.max_rows, p.status);
   const int bp = b / p.nq;  // the sequence whose rows the candidates index
   int ncb = p.cand_count[b];
@@ -382,12 +389,8 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
     set_status(p.status, ST_DEVICE_CHECK);
     ncb = ncb < 0 ? 0 : p.cand_stride;
   }
-  const int e0 = rank * EPC;  // first candidate of this CTA
-
-  for (int i = t; i < EPC / CSA2_BLK; i += RS_NT) {
-    const int cb = e0 / CSA2_BLK + i;
-    s.blocks[i] = cb < ncb ? p.cand[(int64_t)b * p.cand_stride + cb] : -1;
-  }
+  static_assert(EPC / CSA2_BLK <= RS_NT, "one candidate block per thread");
+  if (t < EPC / CSA2_BLK) s.blocks[t] = e0 / CSA2_BLK + t < ncb ? cblk : -1;
   // B fragments: head n = lane / 4 (8 heads = MMA N), this thread's 16
   // contiguous channels [16c, 16c + 16) of the 64, c = lane % 4.  The K axis
   // is permuted identically for A and B so that each thread loads 32
@@ -493,18 +496,23 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int b = blockIdx.y;
+  const int e0 = (rank * BS_NT + threadIdx.x) * BS_KPT;
+  // the block maxima are read without waiting for the count (within the
+  // row's stride, a multiple of 16), so both loads are in flight together
+  const float* src = bm + (int64_t)b * bm_stride + e0;
+  float4 v[BS_KPT / 4];
+#pragma unroll
+  for (int j = 0; j < BS_KPT / 4; j++)
+    v[j] = e0 + 4 * j < bm_stride ? *reinterpret_cast<const float4*>(src + 4 * j)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
   const int C = visible_query(n_rows, b, nq, max_rows, status);
   const int nblk = (C + CSA2_BLK - 1) / CSA2_BLK;
-  const int e0 = (rank * BS_NT + threadIdx.x) * BS_KPT;
   uint32_t key[BS_KPT];
-  const float* src = bm + (int64_t)b * bm_stride + e0;
 #pragma unroll
-  for (int j = 0; j < BS_KPT; j += 4) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (e0 + j < nblk) v = *reinterpret_cast<const float4*>(src + j);
-    const float f[4] = {v.x, v.y, v.z, v.w};
+  for (int j = 0; j < BS_KPT / 4; j++) {
+    const float f[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-    for (int u = 0; u < 4; u++) key[j + u] = (e0 + j + u < nblk) ? float_key(f[u]) : 0u;
+    for (int u = 0; u < 4; u++) key[4 * j + u] = (e0 + 4 * j + u < nblk) ? float_key(f[u]) : 0u;
   }
   cluster_select_topk<BS_NT, BS_KPT>(sm, key, [](int e) { return e; }, k_req,
                                      sel + (int64_t)b * sel_stride, sel_count + b);

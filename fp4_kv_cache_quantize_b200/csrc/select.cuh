@@ -6,24 +6,30 @@
 // towards the lower element index, returned in ascending element order.
 //
 // The k-th largest key is found by narrowing a bracket [lo, hi] of key
-// values round by round, with counting only (no shared-memory atomics: on
-// this GPU a CTA of shared atomics over a few thousand keys costs several
-// microseconds, which is what a histogram-per-pass radix select spends):
-//   * round 0: the candidates' maximum, minimum and number, one warp
-//     reduction (redux.sync) per quantity, then across warps and ranks;
-//   * each further round cuts [lo, hi] into SEL_NB equal bins of key values
-//     (a power-of-two width, so the bin is a subtraction and a shift); every
-//     lane counts its keys inside the bracket into 4-bit fields of packed
-//     64-bit counters, a warp adds its lanes' counts with one redux.sync per
-//     pair of bins, CTA and cluster totals follow; the bin holding the k-th
-//     key becomes the new bracket.  A round ends the search when the bin's
-//     keys are exactly the ones still wanted, or when the bracket holds a
-//     single key value (then the lowest element indices among the keys equal
-//     to it are taken).
-// Cluster exchanges push each CTA's few counters into every rank's shared
-// memory before a cluster barrier (remote stores never wait), so every read
-// after a barrier is local.  One packed prefix scan then places every
-// selected element in element order.
+// values round by round:
+//   * round 0: the candidates' maximum, minimum and number (warp reductions,
+//     then across warps and cluster ranks);
+//   * each counting round cuts [lo, hi] into equal bins of key values (a
+//     power-of-two width: the bin is a subtraction and a shift) and counts
+//     the bracket's keys per bin; the bin holding the k-th largest key
+//     becomes the new bracket.  The first round sees every key: it uses 16
+//     bins, each lane counts into 4-bit fields of one 64-bit register, and a
+//     warp adds its lanes' counters with six shuffles (a reduce-scatter that
+//     leaves one bin's warp total per lane pair) before one shared-memory
+//     atomic per bin.  Later rounds see few keys: 64 bins, one shared atomic
+//     per key in the bracket.
+//   * a round ends the search when the bin's keys are exactly the ones still
+//     wanted, or when the bin is a single key value (the lowest element
+//     indices among the keys equal to it are taken).
+// The code runs once per CTA and every instruction of it is fetched cold
+// (instruction fetch, not arithmetic, bounds this kernel's latency), so all
+// rounds run the same rolled loop body.
+// Cluster exchanges push each CTA's counts into every rank's shared memory
+// before a cluster barrier (remote stores do not wait), so every read after
+// a barrier is local and every rank can work out every rank's share of the
+// result.  The placement needs no further exchange: each rank knows how many
+// selected elements precede it and how many of its keys equal to the
+// threshold it takes, and places its own with one block prefix scan.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -34,21 +40,21 @@ namespace csa2 {
 
 namespace cg = cooperative_groups;
 
-constexpr int SEL_DB0 = 4;             // key bits the first counting round resolves (at best)
-constexpr int SEL_DB = 6;              // ... and every later round
-constexpr int SEL_NB = 1 << SEL_DB;    // bins of a round, at most
+constexpr int SEL_NB = 64;             // bins of a light round
 constexpr int SEL_MAX_RANKS = 16;
 
 template <int NT, int KPT>
 struct SelectSmem {
   static constexpr int NW = NT / 32;
-  uint32_t wcnt[NW][SEL_NB / 2];                 // per-warp counts, bins (2i, 2i+1) as 16-bit halves
-  uint32_t xbuf[2][SEL_MAX_RANKS][SEL_NB / 2];   // per-rank CTA counts, by round parity
+  uint32_t hist[SEL_NB];                         // this CTA's counts of the round
+  uint32_t xbuf[2][SEL_MAX_RANKS][SEL_NB];       // every rank's counts, by round parity
   uint32_t wred[NW][4];                          // round 0: per-warp max, min, count
-  uint32_t cinfo[SEL_MAX_RANKS][4];              // round 0: per-rank max, min, count
-  uint32_t verdict[4];                           // the round's chosen bin, keys above it, keys in it
+  alignas(16) uint32_t cinfo[SEL_MAX_RANKS][4];  // round 0: per-rank max, min, count
+  uint32_t above[SEL_MAX_RANKS];                 // per rank: keys above the bracket
+  uint32_t last[SEL_MAX_RANKS];                  // per rank: keys in the bracket
+  uint32_t verdict[4];
+  uint32_t fin[4];                               // this rank's rule: T, keys == T taken, first output slot
   uint32_t wsum[32];
-  uint32_t info[SEL_MAX_RANKS];                  // placement: per rank (keys > T) << 16 | (keys == T)
 };
 static_assert(sizeof(SelectSmem<256, 4>) % 16 == 0, "keeps what follows 16-byte aligned");
 
@@ -77,68 +83,95 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   return before + x - v;
 }
 
-// One counting round: this CTA's counts of the keys in [lo, lo + span] per
-// bin (key - lo) >> s, bins 0..2^DB-1, pushed as pairs of 16-bit halves into
-// xbuf[par][rank][*] of every rank (the caller's barrier completes them).
-template <int NT, int KPT, int DB>
-__device__ __forceinline__ void count_bins(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
-                                           uint32_t lo, uint32_t span, int s, int par,
-                                           unsigned rank, unsigned ncta,
-                                           cg::cluster_group& cluster) {
-  constexpr int NB = 1 << DB, NP = NB / 16, NW = NT / 32;
-  static_assert(NB >= 16 && NB <= SEL_NB, "bins per round");
+// First counting round: 16 bins of width 2^s over [lo, lo + span], every
+// lane's keys counted into nibbles, warp totals by a shuffle reduce-scatter,
+// one shared atomic per bin and warp into hist.
+template <int N>
+__device__ __forceinline__ void count16(uint32_t* hist, const uint32_t (&key)[N], uint32_t lo,
+                                        uint32_t span, int s) {
+  static_assert(N <= 15, "4-bit per-lane counters");
   constexpr uint32_t FULL = 0xffffffffu;
-  const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-  uint64_t c[NP];
+  const int lane = threadIdx.x & 31;
+  uint64_t c = 0ull;
 #pragma unroll
-  for (int q = 0; q < NP; q++) c[q] = 0ull;
-  bool any = false;
-#pragma unroll
-  for (int j = 0; j < KPT; j++) {
+  for (int j = 0; j < N; j++) {
     const uint32_t d = key[j] - lo;  // keys below lo (and 0) wrap past span
-    if (d <= span) {
-      const uint32_t b = d >> s;
-      const uint64_t inc = 1ull << ((b & 15u) * 4u);
-      if constexpr (NP == 1) {
-        c[0] += inc;
-      } else {
+    if (d <= span) c += 1ull << (((d >> s) & 15u) * 4u);
+  }
+  // nibbles -> bytes: w_i holds bins 4i..4i+3 (at most 15 each)
+  const uint32_t x0 = (uint32_t)c, x1 = (uint32_t)(c >> 32);
+  const uint32_t e0 = x0 & 0x0F0F0F0Fu, o0 = (x0 >> 4) & 0x0F0F0F0Fu;
+  const uint32_t e1 = x1 & 0x0F0F0F0Fu, o1 = (x1 >> 4) & 0x0F0F0F0Fu;
+  const uint32_t w0 = __byte_perm(e0, o0, 0x5140), w1 = __byte_perm(e0, o0, 0x7362);
+  const uint32_t w2 = __byte_perm(e1, o1, 0x5140), w3 = __byte_perm(e1, o1, 0x7362);
+  // lanes with bit 4 clear keep bins 0-7 (w0, w1), the others bins 8-15
+  const bool b4 = lane & 16;
+  uint32_t k0 = b4 ? w2 : w0, k1 = b4 ? w3 : w1;
+  k0 += __shfl_xor_sync(FULL, b4 ? w0 : w2, 16);
+  k1 += __shfl_xor_sync(FULL, b4 ? w1 : w3, 16);
+  // bit 3: one word of 4 bins (bytes; at most 4 x 15 = 60)
+  const bool b3 = lane & 8;
+  uint32_t k = b3 ? k1 : k0;
+  k += __shfl_xor_sync(FULL, b3 ? k0 : k1, 8);
+  // bit 2: two bins as 16-bit halves
+  const bool b2 = lane & 4;
+  const uint32_t lo2 = __byte_perm(k, 0u, 0x4140), hi2 = __byte_perm(k, 0u, 0x4342);
+  uint32_t h = b2 ? hi2 : lo2;
+  h += __shfl_xor_sync(FULL, b2 ? lo2 : hi2, 4);
+  // bit 1: one bin
+  const bool b1 = lane & 2;
+  uint32_t v = b1 ? (h >> 16) : (h & 0xFFFFu);
+  v += __shfl_xor_sync(FULL, b1 ? (h & 0xFFFFu) : (h >> 16), 2);
+  // bit 0: lanes 2i and 2i+1 hold bin i; the pair's sum is the warp total
+  v += __shfl_xor_sync(FULL, v, 1);
+  if ((lane & 1) == 0 && v != 0u) atomicAdd(&hist[lane >> 1], v);
+}
+
+// Later rounds: 64 bins, one shared atomic per key in the bracket.
+template <int N>
+__device__ __forceinline__ void count64(uint32_t* hist, const uint32_t (&key)[N], uint32_t lo,
+                                        uint32_t span, int s) {
 #pragma unroll
-        for (int q = 0; q < NP; q++) c[q] += (b >> 4) == (uint32_t)q ? inc : 0ull;
-      }
-      any = true;
+  for (int j = 0; j < N; j++) {
+    const uint32_t d = key[j] - lo;
+    if (d <= span) atomicAdd(&hist[d >> s], 1u);
+  }
+}
+
+// Warp 0: the bin of the krem-th largest key from per-rank counts
+// xs[r][b] (r < nr); writes (bin, keys above it, keys in it) to verdict.
+template <class Smem>
+__device__ __forceinline__ void find_bin(Smem& sm, const uint32_t (*xs)[SEL_NB], unsigned nr,
+                                         uint32_t krem) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  uint32_t c0 = 0u, c1 = 0u;
+#pragma unroll
+  for (unsigned r = 0; r < SEL_MAX_RANKS; r++) {  // all loads in flight at once
+    if (r < nr) {
+      c0 += xs[r][2 * lane];
+      c1 += xs[r][2 * lane + 1];
     }
   }
-  if (__any_sync(FULL, any)) {
-    // nibbles -> 16-bit halves: word w holds bins 2w (low) and 2w+1 (high)
+  const uint32_t pair = c0 + c1;
+  uint32_t suf = pair;  // keys in bins >= 2 lane
 #pragma unroll
-    for (int h = 0; h < 2 * NP; h++) {
-      const uint32_t x = (uint32_t)(c[h >> 1] >> (32 * (h & 1)));
-      const uint32_t ev = x & 0x0F0F0F0Fu, od = (x >> 4) & 0x0F0F0F0Fu;
-      const uint32_t i01 = __byte_perm(ev, od, 0x5140), i23 = __byte_perm(ev, od, 0x7362);
-      const uint32_t w4[4] = {__byte_perm(i01, 0u, 0x4140), __byte_perm(i01, 0u, 0x4342),
-                              __byte_perm(i23, 0u, 0x4140), __byte_perm(i23, 0u, 0x4342)};
-#pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const uint32_t v = __reduce_add_sync(FULL, w4[u]);
-        if (lane == 0) sm.wcnt[wid][4 * h + u] = v;
-      }
-    }
-  } else if (lane < NB / 2) {
-    sm.wcnt[wid][lane] = 0u;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(FULL, suf, o);
+    if (lane + o < 32) suf += y;
   }
-  __syncthreads();
-  if (t < SEL_NB / 2) {  // this CTA's counts of bins (2t, 2t+1), pushed to every rank
-    uint32_t v = 0u;
-    if (t < NB / 2) {
-#pragma unroll 8
-      for (int w = 0; w < NW; w++) v += sm.wcnt[w][t];
-    }
-    if (ncta > 1) {
-      for (unsigned r = 0; r < ncta; r++) *cluster.map_shared_rank(&sm.xbuf[par][rank][t], r) = v;
-    } else {
-      sm.xbuf[par][0][t] = v;
-    }
+  const uint32_t above_hi = suf - pair;  // bins > 2 lane + 1
+  if (above_hi < krem && above_hi + pair >= krem) {
+    const bool in_hi = above_hi + c1 >= krem;
+    sm.verdict[0] = in_hi ? 2u * lane + 1u : 2u * lane;
+    sm.verdict[1] = in_hi ? above_hi : above_hi + c1;
+    sm.verdict[2] = in_hi ? c1 : c0;
   }
+}
+
+__device__ __forceinline__ int round_shift(uint32_t span, int bits) {
+  const int nbits = 32 - __clz(span);
+  return nbits > bits ? nbits - bits : 0;
 }
 
 // Every thread of every CTA of the cluster calls this with the same k_req.
@@ -152,7 +185,7 @@ template <int NT, int KPT, class IdOf>
 __device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
                                     IdOf id_of, int k_req, int32_t* out, int32_t* out_count,
                                     bool cluster_wide = true) {
-  static_assert(NT >= 64 && NT % 32 == 0, "at least two warps");
+  static_assert(NT >= 64 && NT % 32 == 0, "at least 64 threads");
   static_assert(KPT <= 15, "4-bit per-lane counters");
   static_assert(NT * KPT < 65536, "16-bit packed counts");
   constexpr int NW = NT / 32;
@@ -161,8 +194,13 @@ __device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&ke
   const unsigned rank = cluster_wide ? cluster.block_rank() : 0u;
   const unsigned ncta = cluster_wide ? cluster.num_blocks() : 1u;
   const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  auto csync = [&]() {
+    if (ncta > 1) cluster.sync();
+    else __syncthreads();
+  };
 
   // ---- round 0: maximum, minimum and number of candidates
+  if (t < SEL_NB) sm.hist[t] = 0u;
   {
     uint32_t mx = 0u, mn = FULL, cnt = 0u;
 #pragma unroll
@@ -201,115 +239,132 @@ __device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&ke
         dst[2] = c;
       }
     }
-    if (ncta > 1) cluster.sync();
-    else __syncthreads();
+    csync();
   }
-  uint32_t gmx = 0u, gmn = FULL, gcnt = 0u;
-  for (unsigned r = 0; r < ncta; r++) {
-    gmx = max(gmx, sm.cinfo[r][0]);
-    gmn = min(gmn, sm.cinfo[r][1]);
-    gcnt += sm.cinfo[r][2];
+  uint32_t gmx = 0u, gmn = FULL, gcnt = 0u, cnt_below = 0u;
+#pragma unroll
+  for (unsigned r = 0; r < SEL_MAX_RANKS; r++) {
+    if (r < ncta) {
+      const uint4 ci = *reinterpret_cast<const uint4*>(sm.cinfo[r]);
+      gmx = max(gmx, ci.x);
+      gmn = min(gmn, ci.y);
+      gcnt += ci.z;
+      if (r < rank) cnt_below += ci.z;
+    }
   }
-  const uint32_t k = (uint32_t)(k_req > 0 ? k_req : 0) < gcnt ? (uint32_t)(k_req > 0 ? k_req : 0)
-                                                              : gcnt;
+  const uint32_t kr = (uint32_t)(k_req > 0 ? k_req : 0);
+  const uint32_t k = kr < gcnt ? kr : gcnt;
 
-  // The selection: every key > Tx, then the first keq keys == Tx in element
-  // order (keq = 0 when every key >= Tx + 1 is taken).
-  uint32_t Tx = FULL, keq = 0u;
-  if (k > 0u && k == gcnt) {
-    Tx = gmn - 1u;  // every candidate (gmn >= 1)
-  } else if (k > 0u) {
+  // The result on every rank r: every key > Tx, then the first keq_r keys
+  // == Tx of the rank in element order, placed from output slot off_r.
+  if (k == 0u || k == gcnt) {
+    if (t == 0) {
+      sm.fin[0] = k ? gmn - 1u : FULL;  // every candidate, or none
+      sm.fin[1] = 0u;
+      sm.fin[2] = k ? cnt_below : 0u;
+    }
+    __syncthreads();
+  } else {
     uint32_t lo = gmn, hi = gmx, krem = k;
-    // each round leaves at most 2^(span bits - SEL_DB0 or SEL_DB) key values:
-    // the bracket is a single value after at most 8 rounds
-    for (int round = 0;; round++) {
-      if (lo == hi || round == 12) {  // one key value left: ties by element order
-        Tx = lo;
-        keq = krem;
-        break;
-      }
-      const uint32_t span = hi - lo;
-      const int nbits = 32 - __clz(span);
-      int shift;
+    if (t < SEL_MAX_RANKS) sm.above[t] = 0u;
+    int mode = 0;  // 1: the whole bin; 2: one key value
+    uint32_t nlo = lo, nhi = hi;
+    for (int round = 0; round < 12; round++) {
+      const uint32_t span = hi - lo;  // > 0 here
       const int par = round & 1;
-      // the first round sees every key: fewer bins keep it cheap; later
-      // rounds see few keys and resolve more bits each
+      int s;
       if (round == 0) {
-        const int s = nbits > SEL_DB0 ? nbits - SEL_DB0 : 0;
-        shift = s;
-        count_bins<NT, KPT, SEL_DB0>(sm, key, lo, span, s, par, rank, ncta, cluster);
+        s = round_shift(span, 4);
+        count16<KPT>(sm.hist, key, lo, span, s);
       } else {
-        const int s = nbits > SEL_DB ? nbits - SEL_DB : 0;
-        shift = s;
-        count_bins<NT, KPT, SEL_DB>(sm, key, lo, span, s, par, rank, ncta, cluster);
+        s = round_shift(span, 6);
+        count64<KPT>(sm.hist, key, lo, span, s);
       }
-      if (ncta > 1) cluster.sync();
-      else __syncthreads();
-      // ---- warp 0: totals of bins (2 lane, 2 lane + 1), the bin of the k-th key
-      if (wid == 0) {
-        uint32_t c0 = 0u, c1 = 0u;
-        for (unsigned r = 0; r < ncta; r++) {
-          const uint32_t v = sm.xbuf[par][r][lane];
-          c0 += v & 0xFFFFu;
-          c1 += v >> 16;
+      __syncthreads();
+      if (t < SEL_NB) {  // push this CTA's counts to every rank
+        const uint32_t v = sm.hist[t];
+        sm.hist[t] = 0u;
+        if (ncta > 1) {
+          for (unsigned r = 0; r < ncta; r++) *cluster.map_shared_rank(&sm.xbuf[par][rank][t], r) = v;
+        } else {
+          sm.xbuf[par][0][t] = v;
         }
-        // keys in bins above 2 lane + 1: suffix sum over the higher lanes
-        uint32_t pair = c0 + c1, suf = pair;
+      }
+      csync();
+      if (wid == 0) find_bin(sm, sm.xbuf[par], ncta, krem);
+      __syncthreads();
+      const uint32_t jb = sm.verdict[0], above = sm.verdict[1], inbin = sm.verdict[2];
+      for (int r = wid; r < (int)ncta; r += NW) {  // warp r: rank r's keys above the bin and in it
+        const uint32_t* xr = sm.xbuf[par][r];
+        uint32_t a = (2 * lane > (int)jb ? xr[2 * lane] : 0u) +
+                     (2 * lane + 1 > (int)jb ? xr[2 * lane + 1] : 0u);
+        a = __reduce_add_sync(FULL, a);
+        if (lane == 0) {
+          sm.above[r] += a;
+          sm.last[r] = xr[jb];
+        }
+      }
+      krem -= above;
+      nlo = lo + (jb << s);
+      const uint64_t h64 = (uint64_t)nlo + ((1ull << s) - 1ull);
+      nhi = h64 < (uint64_t)hi ? (uint32_t)h64 : hi;
+      if (inbin == krem) { mode = 1; break; }
+      if (nlo == nhi || round == 11) { mode = 2; break; }  // 32 bits take at most 6 rounds
+      lo = nlo;
+      hi = nhi;
+    }
+    __syncthreads();  // above / last complete
+    {
+      if (wid == 0) {
+        // lane r = rank r.  mode 1: every key of the bin (>= nlo); mode 2:
+        // the first krem keys == nlo in element order (ranks in order)
+        const bool in = lane < (int)ncta;
+        const uint32_t e = in ? sm.last[lane] : 0u, ab = in ? sm.above[lane] : 0u;
+        uint32_t eqi = e;  // inclusive prefix over ranks of the keys in the bin
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_down_sync(FULL, suf, o);
-          if (lane + o < 32) suf += y;
+          const uint32_t y = __shfl_up_sync(FULL, eqi, o);
+          if (lane >= o) eqi += y;
         }
-        const uint32_t above_hi = suf - pair;  // bins > 2 lane + 1
-        if (above_hi < krem && above_hi + pair >= krem) {
-          const bool in_hi = above_hi + c1 >= krem;
-          sm.verdict[0] = in_hi ? 2u * lane + 1u : 2u * lane;
-          sm.verdict[1] = in_hi ? above_hi : above_hi + c1;
-          sm.verdict[2] = in_hi ? c1 : c0;
+        const uint32_t eqb = eqi - e;
+        const uint32_t kq = mode == 1 ? 0u : (krem > eqb ? min(krem - eqb, e) : 0u);
+        const uint32_t sel = ab + (mode == 1 ? e : kq);
+        uint32_t seli = sel;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(FULL, seli, o);
+          if (lane >= o) seli += y;
+        }
+        if (lane == (int)rank) {
+          sm.fin[0] = mode == 1 ? nlo - 1u : nlo;
+          sm.fin[1] = kq;
+          sm.fin[2] = seli - sel;
         }
       }
       __syncthreads();
-      const uint32_t jb = sm.verdict[0], above = sm.verdict[1], inbin = sm.verdict[2];
-      krem -= above;
-      const uint32_t nlo = lo + (jb << shift);
-      const uint64_t nhi = (uint64_t)nlo + ((1ull << shift) - 1ull);
-      if (inbin == krem) {  // the whole bin: every key >= nlo
-        Tx = nlo - 1u;
-        keq = 0u;
-        break;
-      }
-      lo = nlo;
-      hi = nhi < (uint64_t)hi ? (uint32_t)nhi : hi;
     }
   }
 
-  // ---- placement: every key > Tx, then the first keq keys == Tx
+  // ---- placement: every key > Tx, then the first keq keys == Tx of this rank
+  const uint32_t Tx = sm.fin[0], keq = sm.fin[1], out_off = sm.fin[2];
   uint32_t gt = 0u, eq = 0u;
 #pragma unroll
   for (int j = 0; j < KPT; j++) {
     gt += key[j] > Tx;
-    eq += key[j] == Tx;
+    eq += key[j] == Tx && key[j] != 0u;
   }
   uint32_t tot;
   const uint32_t excl = block_excl_scan<NT>((gt << 16) | eq, sm.wsum, tot);
-  uint32_t gt_before = 0u, eq_before = 0u;  // over the cluster ranks below this one
-  if (ncta > 1) {
-    if (t < (int)ncta) *cluster.map_shared_rank(&sm.info[rank], t) = tot;
-    cluster.sync();  // the last cluster barrier: no remote access after it
-    for (unsigned r = 0; r < rank; r++) {
-      gt_before += sm.info[r] >> 16;
-      eq_before += sm.info[r] & 0xFFFFu;
-    }
-  }
   if (k > 0u) {
-    const uint32_t eq_rank = eq_before + (excl & 0xFFFFu);  // keys == Tx before this thread
+    const uint32_t eq_rank = excl & 0xFFFFu;  // keys == Tx of this rank before this thread
     const uint32_t take_eq = keq > eq_rank ? min(keq - eq_rank, eq) : 0u;
-    uint32_t pos = gt_before + (excl >> 16) + min(keq, eq_rank), taken = 0u;
+    uint32_t pos = out_off + (excl >> 16) + min(keq, eq_rank), taken = 0u;
     const int e0 = ((int)rank * NT + t) * KPT;
 #pragma unroll
     for (int j = 0; j < KPT; j++) {
-      const bool pick = key[j] > Tx || (key[j] == Tx && taken < take_eq);
-      if (key[j] == Tx && pick) taken++;
+      const bool tie = key[j] == Tx && key[j] != 0u;
+      const bool pick = key[j] > Tx || (tie && taken < take_eq);
+      if (tie && pick) taken++;
       if (pick) out[pos++] = id_of(e0 + j);
     }
   }

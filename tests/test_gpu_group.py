@@ -119,6 +119,23 @@ def test_group_ragged_paged_no_pool(lib, orc):
     compare_group(orc, dw, run_group(lib, dw))
 
 
+def test_group_query_magnitudes(lib, orc):
+    """Main queries whose heads span bf16's range, from 1e-6 to 1e5 (beyond
+    fp16's 65,504) and all-zero heads: the attention must match the oracle
+    with no overflow and no loss of small queries."""
+    wl = synth.config(0)
+    q = synth.bf16_bits_to_f32(wl.q).astype(np.float64)
+    scale = np.array([1e-6, 3e-5, 1e-3, 0.25, 1.0, 7.0, 100.0, 2e3,
+                      3e4, 6.5e4, 1e5, 1e5, 0.0, 1.0, 1e-6, 5e4])
+    for l in range(wl.L):
+        sc = np.roll(scale, l)
+        q[l] *= sc[None, :, None]
+    wl.q = synth.to_bf16_bits(q.astype(np.float32))
+    assert np.abs(synth.bf16_bits_to_f32(wl.q)).max() > 65504.0
+    dw = DeviceWorkload(lib, wl, orc)
+    compare_group(orc, dw, run_group(lib, dw))
+
+
 def test_group_rejects_leading_reuse(lib, orc):
     wl = synth.make("bad", seed=3, B=1, n_rows=[100], modes=[REUSE, FULL])
     dw = DeviceWorkload(lib, wl, orc)

@@ -94,6 +94,7 @@ def run_and_check(lib, orc, n_rows, Q, modes, swa_len, pool_blocks, seed, paged=
 @pytest.mark.parametrize("Q,n_rows,swa_len", [
     (2, [20000, 9001], [129, 40]),
     (3, [12000, 700], [130, 3]),
+    (4, [15000, 3000], [131, 77]),  # the draft count the benchmark's multi-query line times
     (8, [9000, 2050], [135, 100]),
     (20, [3000, 10], [147, 5]),     # three scan passes; early queries of b=1 see nothing
     (64, [2500], [191]),            # chunked prefill: eight scan passes
