@@ -326,13 +326,15 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   // ---- S^T = K . Q'^T (one thread issues 32 MMAs of K = 16)
   if (nk > 0 && t == 0) {
     tc_fence_after();
-    const uint32_t a0 = smem_u32(s.tile), b0 = smem_u32(s.q);
+    // descriptors advance by adding (byte offset >> 4) to the start-address
+    // field (every operand lies below 256 KB, so the field never carries)
+    const uint64_t da = sdesc_k128(smem_u32(s.tile)), db = sdesc_k128(smem_u32(s.q));
 #pragma unroll 1
-    for (int kb = 0; kb < 8; kb++)
-#pragma unroll
-      for (int sub = 0; sub < 4; sub++)
-        umma_bf16(tmem, sdesc_k128(a0 + kb * TA_KB + 32 * sub), sdesc_k128(b0 + kb * 2048 + 32 * sub),
-                  TA_IDESC_QK, (kb | sub) != 0);
+    for (int i = 0; i < 32; i++) {  // K = 512 in 32 steps: block kb = i / 4, 32-byte step i % 4
+      const uint32_t kb = (uint32_t)i >> 2, sub = (uint32_t)i & 3;
+      umma_bf16(tmem, da + ((kb * TA_KB + 32 * sub) >> 4), db + ((kb * 2048 + 32 * sub) >> 4),
+                TA_IDESC_QK, i != 0);
+    }
     umma_commit(&s.mbar);
   }
   float* sS = reinterpret_cast<float*>(s.raw);  // logits [head][key], log2 units
@@ -393,12 +395,12 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   // ---- O^T = V^T . P^T: four channel blocks of 128, K = 128 keys in 8 steps
   if (nk > 0 && t == 0) {
     tc_fence_after();
-    const uint32_t a0 = smem_u32(s.tile), b0 = smem_u32(s.p);
+    const uint64_t da = sdesc_mn128(smem_u32(s.tile), TA_KB, 1024), db = sdesc_k128(smem_u32(s.p));
 #pragma unroll 1
-    for (int i = 0; i < 32; i++) {
-      const int cb = i >> 3, ks = i & 7;
-      umma_bf16(tmem + TA_O_COL + 16 * cb, sdesc_mn128(a0 + cb * 2 * TA_KB + ks * 2048, TA_KB, 1024),
-                sdesc_k128(b0 + (ks >> 2) * 2048 + (ks & 3) * 32), TA_IDESC_PV, ks > 0);
+    for (int i = 0; i < 32; i++) {  // channel block cb = i / 8, 16 keys ks = i % 8
+      const uint32_t cb = (uint32_t)i >> 3, ks = (uint32_t)i & 7;
+      umma_bf16(tmem + TA_O_COL + 16 * cb, da + ((cb * 2 * TA_KB + ks * 2048) >> 4),
+                db + (((ks >> 2) * 2048 + (ks & 3) * 32) >> 4), TA_IDESC_PV, ks > 0);
     }
     umma_commit(&s.mbar);
   }

@@ -157,6 +157,7 @@ static ScanParams scan_params(const csa2_kv_view* kv, const float* w, const Inde
   p.nq_pass = nq;
   p.tail = 0;
   p.status = ws.status;
+  p.sched = ws.status + CSA2_WS_SCHED_WORD;  // the scan's tile counters in the header
   return p;
 }
 

@@ -54,7 +54,9 @@ struct ScanCfg {
     uint8_t a[SC_STAGES][SC_A_BYTES];
     uint8_t b[SC_STAGES][B_BYTES];
     uint64_t full[SC_STAGES], empty[SC_STAGES];
-    uint64_t tfull[ACC], tempty[ACC], done;
+    uint64_t tfull[ACC], tempty[ACC], tinfo[ACC], done;
+    int32_t tile[SC_STAGES];  // the tile each stage holds (-1: no more tiles)
+    int32_t acc_tile[ACC];    // the tile each accumulator holds (-1: no more tiles)
     uint32_t tmem_base;
     int abort;
     // N = 64 (two batches of TMEM loads per tile): each epilogue warp's copy
@@ -125,6 +127,7 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
     for (int i = 0; i < ACC; i++) {
       mbar_init(&s.tfull[i], 1);
       mbar_init(&s.tempty[i], Cfg::EPI_WARPS * 32);
+      mbar_init(&s.tinfo[i], 1);
     }
     mbar_init(&s.done, 1);
     s.abort = 0;
@@ -150,7 +153,15 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
       int stage = 0, cur_b = -1, C = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
       const uint64_t stream_once = l2_policy_evict_first();  // indexer K is read once per step
-      for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+      // Tiles are handed out by a counter in the workspace header, one at a
+      // time, so that CTAs that run faster take more of them (a fixed
+      // interleave leaves a tail of slow CTAs); the next tile is requested
+      // while the current one is issued.
+      uint32_t next = atomicAdd(p.sched, 1u);
+      while (true) {
+        const int64_t g = next;
+        if (g >= total) break;
+        next = atomicAdd(p.sched, 1u);
         const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
         if (b != cur_b) {
           C = visible_rows(p.n_rows, b, p.max_rows, p.status);
@@ -162,6 +173,7 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
           set_status(p.status, ST_TIMEOUT);
           break;
         }
+        s.tile[stage] = (int32_t)g;
         const int pos0 = t * SC_TILE;
         const int32_t y0 = box_row(p, b, pos0);
         const int32_t y1 = pos0 + SC_BOX < C - p.tail ? box_row(p, b, pos0 + SC_BOX) : y0;
@@ -176,6 +188,18 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
           phase ^= 1u;
         }
       }
+      // end of the tiles: a stage that carries no data, only the marker
+      if (!*abort) {
+        if (mbar_wait(&s.empty[stage], phase ^ 1u, abort)) {
+          // this stage's earlier copy has been consumed, so it has landed
+          issued &= ~(1u << stage);
+          s.tile[stage] = -1;
+          mbar_arrive(&s.full[stage]);
+        } else {
+          s.abort = 1;
+          set_status(p.status, ST_TIMEOUT);
+        }
+      }
       // Drain: every issued copy lands before the CTA may exit.
       for (int i = 0; i < SC_STAGES; i++)
         if ((issued >> i) & 1u)
@@ -184,21 +208,19 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------------------------- MMA issuer
-      int stage = 0, acc = 0, cur_b = -1, C = 0;
+      int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
-        const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
-        if (b != cur_b) {
-          C = visible_rows(p.n_rows, b, p.max_rows, nullptr);
-          cur_b = b;
-        }
-        if (t * SC_TILE >= C - p.tail) continue;
+      while (true) {
         if (!mbar_wait(&s.full[stage], phase, abort) ||
             !mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort)) {
           s.abort = 1;
           set_status(p.status, ST_TIMEOUT);
           break;
         }
+        const int32_t tile = s.tile[stage];
+        s.acc_tile[acc] = tile;
+        mbar_arrive(&s.tinfo[acc]);  // the epilogue learns the tile (or the end)
+        if (tile < 0) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(s.a[stage]), b_addr = smem_u32(s.b[stage]);
         const uint32_t d = tmem + (uint32_t)(acc * N);
@@ -232,7 +254,14 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
     uint32_t acc_phase = 0;
     int cur_b = -1, C = 0, w_b = -1, w_t0 = -1;
     float wr[QPB][CSA2_HI];
-    for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+    while (true) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.tinfo[acc], acc_phase, abort))) {
+        s.abort = 1;
+        set_status(p.status, ST_TIMEOUT);
+        break;
+      }
+      const int64_t g = s.acc_tile[acc];
+      if (g < 0) break;
       const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
       if (b != cur_b) {
         C = visible_rows(p.n_rows, b, p.max_rows, nullptr);  // the last query's view
@@ -245,7 +274,6 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
           __syncwarp();
         }
       }
-      if (t * SC_TILE >= C - p.tail) continue;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.tfull[acc], acc_phase, abort));
       if (!ok) {
         s.abort = 1;
@@ -325,6 +353,16 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
+  // The last CTA to finish returns the tile counter to zero for the next
+  // launch (every CTA's producer has stopped taking tiles by then).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      p.sched[0] = 0u;
+      p.sched[1] = 0u;
+      __threadfence();
+    }
+  }
 }
 
 // ------------------------------------------------- rescore + Top-k select
@@ -362,57 +400,20 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int RS_NT>
-__global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescoreParams p) {
-  constexpr int EPC = RS_EPC;  // candidates per CTA
-  constexpr int RS_KPT = RS_EPC / RS_NT;
-  using RescoreSmem = csa2::RescoreSmem<RS_NT>;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  RescoreSmem& s = *reinterpret_cast<RescoreSmem*>(smem_raw);
-  pdl_launch_dependents();
-  pdl_wait();  // the candidate blocks come from the previous kernel
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int b = blockIdx.y;
-  const RescoreJob job = p.job[blockIdx.z];
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int e0 = rank * EPC;  // first candidate of this CTA
-  // the candidate blocks are read without waiting for their count (within
-  // the list's stride), so both loads are in flight together
-  int cblk = -1;
-  if (t < EPC / CSA2_BLK && e0 / CSA2_BLK + t < p.cand_stride)
-    cblk = p.cand[(int64_t)b * p.cand_stride + e0 / CSA2_BLK + t];
-  const int C = visible_query(p.n_rows, b, p.nq, p.max_rows, p.status);
-  const int bp = b / p.nq;  // the sequence whose rows the candidates index
-  int ncb = p.cand_count[b];
-  if (ncb < 0 || ncb > p.cand_stride) {
-    set_status(p.status, ST_DEVICE_CHECK);
-    ncb = ncb < 0 ? 0 : p.cand_stride;
-  }
-  static_assert(EPC / CSA2_BLK <= RS_NT, "one candidate block per thread");
-  if (t < EPC / CSA2_BLK) s.blocks[t] = e0 / CSA2_BLK + t < ncb ? cblk : -1;
-  // B fragments: head n = lane / 4 (8 heads = MMA N), this thread's 16
-  // contiguous channels [16c, 16c + 16) of the 64, c = lane % 4.  The K axis
-  // is permuted identically for A and B so that each thread loads 32
-  // contiguous bytes of a row; a dot product does not depend on K order.
-  const int c = lane & 3, grp = lane >> 2;
-  uint32_t bq[8];
-  {
-    const uint4* qp = reinterpret_cast<const uint4*>(job.q_idx + ((int64_t)b * CSA2_HI + grp) *
-                                                                     CSA2_DI + 16 * c);
-    const uint4 q0 = __ldg(qp), q1 = __ldg(qp + 1);
-    bq[0] = q0.x; bq[1] = q0.y; bq[2] = q0.z; bq[3] = q0.w;
-    bq[4] = q1.x; bq[5] = q1.y; bq[6] = q1.z; bq[7] = q1.w;
-  }
-  const float w0 = __ldg(job.w + b * CSA2_HI + 2 * c), w1 = __ldg(job.w + b * CSA2_HI + 2 * c + 1);
-  __syncthreads();
-
-  // Score 16 candidates per MMA: rows grp and grp + 8 of a group.  A warp
-  // issues the row loads of RS_GB groups before their MMAs, so that several
-  // gathered rows are in flight per lane.
-  constexpr int NW = RS_NT / 32;
-  constexpr int GPW = EPC / 16 / NW;  // groups per warp
+// Scores this CTA's RS_EPC candidates (positions of blocks[0..RS_EPC/8),
+// -1 = none) against one job's indexer query into keys[] (0 = not a
+// candidate).  16 candidates per MMA: rows grp and grp + 8 of a group; a warp
+// issues the row loads of RS_GB groups before their MMAs, so that several
+// gathered rows are in flight per lane.
+template <int NT>
+__device__ __forceinline__ void score_candidates(const RescoreParams& p, const int32_t* blocks,
+                                                 uint32_t* keys, int bp, int C,
+                                                 const uint32_t (&bq)[8], float w0, float w1) {
+  constexpr int NW = NT / 32;
+  constexpr int GPW = RS_EPC / 16 / NW;  // groups per warp
   constexpr int GB = GPW < RS_GB ? GPW : RS_GB;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = lane & 3, grp = lane >> 2;
   for (int gb = 0; gb < GPW; gb += GB) {
     uint32_t av[GB][2][8];
     bool valid[GB][2];
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
 #pragma unroll
       for (int h = 0; h < 2; h++) {
         const int e = g * 16 + grp + 8 * h;  // candidate index within this CTA
-        const int blk = s.blocks[e / CSA2_BLK];
+        const int blk = blocks[e / CSA2_BLK];
         const int pos = blk * CSA2_BLK + (e % CSA2_BLK);
         int64_t row = -1;
         valid[u][h] = blk >= 0 && pos < C;
@@ -461,11 +462,64 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
       s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
       s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
       if (c == 0) {
-        s.keys[g * 16 + grp] = valid[u][0] ? float_key(s0) : 0u;
-        s.keys[g * 16 + grp + 8] = valid[u][1] ? float_key(s1) : 0u;
+        keys[g * 16 + grp] = valid[u][0] ? float_key(s0) : 0u;
+        keys[g * 16 + grp + 8] = valid[u][1] ? float_key(s1) : 0u;
       }
     }
   }
+}
+
+// B fragments of one job's indexer query: head n = lane / 4 (8 heads = MMA
+// N), this thread's 16 contiguous channels [16c, 16c + 16) of the 64,
+// c = lane % 4.  The K axis is permuted identically for A and B so that each
+// thread loads 32 contiguous bytes of a row; a dot product does not depend on
+// K order.  The query and weights are inputs: read before the wait.
+__device__ __forceinline__ void job_query(const RescoreJob& job, int b, uint32_t (&bq)[8],
+                                          float& w0, float& w1) {
+  const int lane = threadIdx.x & 31, c = lane & 3, grp = lane >> 2;
+  const uint4* qp =
+      reinterpret_cast<const uint4*>(job.q_idx + ((int64_t)b * CSA2_HI + grp) * CSA2_DI + 16 * c);
+  const uint4 q0 = __ldg(qp), q1 = __ldg(qp + 1);
+  bq[0] = q0.x; bq[1] = q0.y; bq[2] = q0.z; bq[3] = q0.w;
+  bq[4] = q1.x; bq[5] = q1.y; bq[6] = q1.z; bq[7] = q1.w;
+  w0 = __ldg(job.w + b * CSA2_HI + 2 * c);
+  w1 = __ldg(job.w + b * CSA2_HI + 2 * c + 1);
+}
+
+template <int RS_NT>
+__global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescoreParams p) {
+  constexpr int EPC = RS_EPC;  // candidates per CTA
+  constexpr int RS_KPT = RS_EPC / RS_NT;
+  using RescoreSmem = csa2::RescoreSmem<RS_NT>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RescoreSmem& s = *reinterpret_cast<RescoreSmem*>(smem_raw);
+  pdl_launch_dependents();
+  const int b = blockIdx.y;
+  const RescoreJob job = p.job[blockIdx.z];
+  uint32_t bq[8];
+  float w0, w1;
+  job_query(job, b, bq, w0, w1);
+  pdl_wait();  // the candidate blocks come from the previous kernel
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int t = threadIdx.x;
+  const int e0 = rank * EPC;  // first candidate of this CTA
+  // the candidate blocks are read without waiting for their count (within
+  // the list's stride), so both loads are in flight together
+  int cblk = -1;
+  if (t < EPC / CSA2_BLK && e0 / CSA2_BLK + t < p.cand_stride)
+    cblk = p.cand[(int64_t)b * p.cand_stride + e0 / CSA2_BLK + t];
+  const int C = visible_query(p.n_rows, b, p.nq, p.max_rows, p.status);
+  const int bp = b / p.nq;  // the sequence whose rows the candidates index
+  int ncb = p.cand_count[b];
+  if (ncb < 0 || ncb > p.cand_stride) {
+    set_status(p.status, ST_DEVICE_CHECK);
+    ncb = ncb < 0 ? 0 : p.cand_stride;
+  }
+  static_assert(EPC / CSA2_BLK <= RS_NT, "one candidate block per thread");
+  if (t < EPC / CSA2_BLK) s.blocks[t] = e0 / CSA2_BLK + t < ncb ? cblk : -1;
+  __syncthreads();
+  score_candidates<RS_NT>(p, s.blocks, s.keys, bp, C, bq, w0, w1);
   __syncthreads();
 
   uint32_t key[RS_KPT];

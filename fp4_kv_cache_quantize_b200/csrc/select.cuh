@@ -181,10 +181,12 @@ __device__ __forceinline__ int round_shift(uint32_t span, int bits) {
 // out[k..k_req) = -1 and *out_count = k (rank 0 writes the last two).
 // With cluster_wide = false the calling CTA selects on its own (rank 0 of a
 // one-CTA selection) even inside a larger cluster.
-template <int NT, int KPT, class IdOf>
-__device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
-                                    IdOf id_of, int k_req, int32_t* out, int32_t* out_count,
-                                    bool cluster_wide = true) {
+// cluster_select_emit: the same selection, handing each selected element to
+// emit(output slot, id) instead of writing an array; returns k.
+template <int NT, int KPT, class IdOf, class Emit>
+__device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
+                                        IdOf id_of, int k_req, Emit emit,
+                                        bool cluster_wide = true) {
   static_assert(NT >= 64 && NT % 32 == 0, "at least 64 threads");
   static_assert(KPT <= 15, "4-bit per-lane counters");
   static_assert(NT * KPT < 65536, "16-bit packed counts");
@@ -365,12 +367,22 @@ __device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&ke
       const bool tie = key[j] == Tx && key[j] != 0u;
       const bool pick = key[j] > Tx || (tie && taken < take_eq);
       if (tie && pick) taken++;
-      if (pick) out[pos++] = id_of(e0 + j);
+      if (pick) emit((int)pos++, id_of(e0 + j));
     }
   }
+  return k;
+}
+
+template <int NT, int KPT, class IdOf>
+__device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
+                                    IdOf id_of, int k_req, int32_t* out, int32_t* out_count,
+                                    bool cluster_wide = true) {
+  const uint32_t k = cluster_select_emit(
+      sm, key, id_of, k_req, [out](int pos, int id) { out[pos] = id; }, cluster_wide);
+  const unsigned rank = cluster_wide ? cg::this_cluster().block_rank() : 0u;
   if (rank == 0) {
-    for (int i = (int)k + t; i < k_req; i += NT) out[i] = -1;
-    if (t == 0 && out_count) *out_count = (int32_t)k;
+    for (int i = (int)k + (int)threadIdx.x; i < k_req; i += NT) out[i] = -1;
+    if (threadIdx.x == 0 && out_count) *out_count = (int32_t)k;
   }
 }
 
