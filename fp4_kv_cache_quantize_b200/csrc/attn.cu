@@ -44,6 +44,7 @@ struct AttnSmem {
   __half p[CSA2_H * AT_CH];    // swizzled rows of 128 B
   float s[CSA2_H][AT_CH + 4];
   float m[CSA2_H], l[CSA2_H], alpha[CSA2_H];
+  uint32_t qmax[CSA2_H][2];  // per head, the two warps' largest |q| (bf16 bits)
   int64_t row[AT_CH];
 };
 
@@ -132,30 +133,52 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
     if (t == 0) L.idx_copy_count[b] = L.idx_count[b];
   }
 
-  // Q (bf16) is loaded now and converted to fp16 (|q| < 65504 required) into
-  // swizzled rows once the first chunk's gathers are in flight.
+  // Q (bf16) is loaded now and converted to fp16, each head scaled by a power
+  // of two (q_pow2_exponent) that is undone on its logits, into swizzled rows
+  // once the first chunk's gathers are in flight.  Chunk i = t + u AT_NT
+  // belongs to head i / 64: warps 2h' and 2h' + 1 hold head h' + 2u.
   constexpr int QV = (CSA2_H * CSA2_D / 8) / AT_NT;
+  static_assert(AT_NT == 128 && QV * 2 == CSA2_H, "two warps per head and chunk set");
   uint4 qv[QV];
   {
     const uint4* qg = reinterpret_cast<const uint4*>(L.q + (int64_t)b * CSA2_H * CSA2_D);
 #pragma unroll
     for (int u = 0; u < QV; u++) qv[u] = __ldg(qg + t + u * AT_NT);
+#pragma unroll
+    for (int u = 0; u < QV; u++) {
+      const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+      uint32_t mx = 0u;
+#pragma unroll
+      for (int k = 0; k < 4; k++) mx = max(mx, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+      mx = __reduce_max_sync(0xffffffffu, mx);
+      if (lane == 0) s.qmax[(t >> 6) + 2 * u][warp & 1] = mx;  // read after a barrier
+    }
   }
   bool q_ready = false;
+  float ls1[2], ls2[2];  // logit factors of heads g and g + 8
   auto store_q = [&]() {
 #pragma unroll
     for (int u = 0; u < QV; u++) {
       const int i = t + u * AT_NT;  // 16-byte chunk of 8 channels
       const int row = i >> 6, ch = i & 63;
+      const int e = q_pow2_exponent(max(s.qmax[row][0], s.qmax[row][1]));
+      const float f1 = pow2i(e / 2), f2 = pow2i(e - e / 2);
       const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
       uint32_t o4[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) {
         const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
-        o4[k] = h2_bits(__floats2half2_rn(lo, hi));
+        o4[k] = h2_bits(__floats2half2_rn(lo * f1 * f2, hi * f1 * f2));
       }
       *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(s.q) + sw1024(row, ch)) =
           make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; j++) {
+      const int h = g + 8 * j;
+      const int e = q_pow2_exponent(max(s.qmax[h][0], s.qmax[h][1]));
+      ls1[j] = pow2i(-(e / 2));
+      ls2[j] = p.scale_log2 * pow2i(-(e - e / 2));
     }
     q_ready = true;
   };
@@ -283,10 +306,10 @@ __global__ void __launch_bounds__(AT_NT, 2) attn_decode_kernel(const AttnParams 
       for (int nt = 0; nt < 2; nt++) {
         const int key = warp * 16 + nt * 8 + 2 * tig;
         const bool v0 = s.row[key] >= 0, v1 = s.row[key + 1] >= 0;
-        s.s[g][key] = v0 ? acc[nt][0] * p.scale_log2 : -INFINITY;
-        s.s[g][key + 1] = v1 ? acc[nt][1] * p.scale_log2 : -INFINITY;
-        s.s[g + 8][key] = v0 ? acc[nt][2] * p.scale_log2 : -INFINITY;
-        s.s[g + 8][key + 1] = v1 ? acc[nt][3] * p.scale_log2 : -INFINITY;
+        s.s[g][key] = v0 ? acc[nt][0] * ls1[0] * ls2[0] : -INFINITY;
+        s.s[g][key + 1] = v1 ? acc[nt][1] * ls1[0] * ls2[0] : -INFINITY;
+        s.s[g + 8][key] = v0 ? acc[nt][2] * ls1[1] * ls2[1] : -INFINITY;
+        s.s[g + 8][key + 1] = v1 ? acc[nt][3] * ls1[1] * ls2[1] : -INFINITY;
       }
     }
     __syncthreads();

@@ -24,9 +24,11 @@
 // the MMA reads.  The softmax runs on the S^T accumulator (one thread per
 // key); P^T in fp16 is the second MMA's B operand.  The five partial results
 // (normalised O in fp16, max and sum per head) are pushed through
-// distributed shared memory to the CTA owning each 128-channel block, one
-// cluster barrier, and the owners merge them with log-sum-exp weights and
-// write the bf16 output: no partials go through global memory.
+// distributed shared memory to the CTA owning each 128-channel block with
+// asynchronous stores counted on the owner's mbarrier (no cluster barrier
+// at the end: an owner waits only for its own 5 x 4,224 bytes), and the
+// owners merge them with log-sum-exp weights and write the bf16 output: no
+// partials go through global memory.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -72,11 +74,15 @@ struct TaSmem {
   int64_t row[TA_KEYS];
   float scl1[CSA2_H], scl2[CSA2_H];        // logit = acc * scl1 * scl2 (log2 units)
   float m[CSA2_H], lsum[CSA2_H], linv[CSA2_H];
-  float2 ml[TA_CTAS][CSA2_H];              // (max, sum) per source CTA, at the owners
+  alignas(16) float2 ml[TA_CTAS][CSA2_H];  // (max, sum) per source CTA, at the owners
   alignas(16) float wts[TA_CTAS][CSA2_H];
   uint64_t mbar;
+  uint64_t rbar;  // an owner's partials have arrived (TA_RECV_BYTES)
   uint32_t tmem_base;
 };
+// bytes each owner receives: per source CTA, 128 channels x 16 heads of fp16
+// O and 16 (max, sum) pairs
+constexpr uint32_t TA_RECV_BYTES = TA_CTAS * (128 * CSA2_H * 2 + CSA2_H * 8);
 constexpr size_t TA_SMEM = sizeof(TaSmem) + 1024;
 
 __device__ __forceinline__ int64_t ta_kv_row(const AttnParams& p, int b, int pos) {
@@ -93,8 +99,6 @@ __device__ __forceinline__ int64_t ta_kv_row(const AttnParams& p, int b, int pos
 
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// 2^e as a float, e in [-126, 127]
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
 // Byte offset of 16-byte chunk cc (0..7) of row r in a 128-byte-swizzled block.
 __device__ __forceinline__ uint32_t sw_off(int r, int cc) {
@@ -118,8 +122,12 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
 
   if (t == 0) {
     mbar_init(&s.mbar, 1);
+    mbar_init(&s.rbar, 1);
     fence_mbar_init();
   }
+  // every CTA's receive barrier is initialised before any partial is sent:
+  // the cluster barrier that orders this completes long before the sends
+  cluster_arrive_release();
   if (warp == 0) {
     tmem_alloc(&s.tmem_base, TA_TMEM_COLS);
     tmem_relinquish();
@@ -141,40 +149,50 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
 
   // ---- this CTA's keys.  b runs over sequences x queries: query tq of
   // sequence bp sees the sequence's entries minus the drafts after it, and
-  // the window rows that end at its own entry.
+  // the window rows that end at its own entry.  Threads r and r + 128 both
+  // resolve key r's row (from the same index) and copy half of it each, so
+  // no thread waits for another before its copies start.
   const int bp = b / p.nq, tq = b - bp * p.nq, later = p.nq - 1 - tq;
+  const int r = t & (TA_KEYS - 1), half = t >> 7;
+  const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
+  const int kt = c * TA_KEYS + r;
   // this thread's index, read before the counts arrive (within the index
   // array's stride either way): the three loads are in flight together
-  const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
-  const int kt = c * TA_KEYS + t;
-  const int pos_t = !window && t < TA_KEYS && kt < p.idx_stride ? __ldg(idx + kt) : -1;
+  const int pos_t = !window && kt < p.idx_stride ? __ldg(idx + kt) : -1;
   int C = p.n_rows[bp];
   if (C < 0 || C > p.max_rows) {
     if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
     C = C < 0 ? 0 : p.max_rows;
   }
   C = C - later < 0 ? 0 : C - later;
-  int nk;  // candidate keys of this CTA: keys j < nk
-  const uint8_t* wbase = nullptr;
+  int nk;          // candidate keys of this CTA: keys j < nk
+  int64_t row = -1;  // key r's row of the cache (or of the window), -1: none
   if (!window) {
     int n_idx = L.idx_count[b];
     if (n_idx < 0 || n_idx > p.idx_stride) {
       if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
       n_idx = n_idx < 0 ? 0 : p.idx_stride;
     }
-    const int k0 = c * TA_KEYS;
-    nk = min(max(n_idx - k0, 0), TA_KEYS);
-    if (L.idx_copy) {  // Reuse layer: publish the indices it used
-      if (t < TA_KEYS && kt < p.idx_stride) L.idx_copy[(int64_t)b * p.idx_stride + kt] = pos_t;
+    nk = min(max(n_idx - c * TA_KEYS, 0), TA_KEYS);
+    if (L.idx_copy && half == 0) {  // Reuse layer: publish the indices it used
+      if (kt < p.idx_stride) L.idx_copy[(int64_t)b * p.idx_stride + kt] = pos_t;
       if (c == 0 && t == 0) L.idx_copy_count[b] = L.idx_count[b];
     }
-    if (t < TA_KEYS) {
-      int64_t row = -1;
-      if (t < nk) {
-        if (pos_t >= 0 && pos_t < C) row = ta_kv_row(p, bp, pos_t);
-        if (row < 0) set_status(p.status, ST_DEVICE_CHECK);
+    if (r < nk) {
+      if (pos_t >= 0 && pos_t < C) row = ta_kv_row(p, bp, pos_t);
+      if (row < 0 && half == 0) set_status(p.status, ST_DEVICE_CHECK);
+    }
+    if (row >= 0) {  // 16 code chunks and 2 scale chunks: 9 per thread
+      const uint8_t* cg_ = p.codes + row * (CSA2_D / 2);
+      const uint8_t* sg_ = p.scales + row * (CSA2_D / 16);
+#pragma unroll 1
+      for (int part = 9 * half; part < 9 * half + 9; part++) {
+        if (part < 16)
+          cp_async16(s.raw + r * TA_CODE_LD + 16 * part, cg_ + 16 * part);
+        else
+          cp_async16(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * (part - 16),
+                     sg_ + 16 * (part - 16));
       }
-      s.row[t] = row;
     }
   } else {
     int n_win = p.swa_len[bp];
@@ -185,34 +203,15 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     const int win_end = n_win - later < 0 ? 0 : n_win - later;
     const int win_lo = win_end > CSA2_W ? win_end - CSA2_W : 0;
     nk = win_end - win_lo;
-    wbase = L.swa + ((int64_t)bp * p.swa_rows + win_lo) * CSA2_D;
-    if (t < TA_KEYS) s.row[t] = t < nk ? (int64_t)t : -1;
-  }
-  __syncthreads();
-
-  // ---- gather the rows (16-byte asynchronous copies)
-  if (nk > 0) {
-    if (!window) {
+    if (r < nk) {  // 32 chunks of 16 E4M3 values: 16 per thread
+      row = r;
+      const uint8_t* wr = L.swa + ((int64_t)bp * p.swa_rows + win_lo + r) * CSA2_D;
 #pragma unroll 1
-      for (int i = t; i < TA_KEYS * 18; i += TA_NT) {
-        const int r = i / 18, part = i - 18 * r;
-        const int64_t row = s.row[r];
-        if (row >= 0) {
-          if (part < 16)
-            cp_async16(s.raw + r * TA_CODE_LD + 16 * part, p.codes + row * (CSA2_D / 2) + 16 * part);
-          else
-            cp_async16(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * (part - 16),
-                       p.scales + row * (CSA2_D / 16) + 16 * (part - 16));
-        }
-      }
-    } else {
-#pragma unroll 1
-      for (int i = t; i < TA_KEYS * 32; i += TA_NT) {
-        const int r = i >> 5, part = i & 31;
-        if (s.row[r] >= 0) cp_async16(s.raw + r * TA_WIN_LD + 16 * part, wbase + r * CSA2_D + 16 * part);
-      }
+      for (int part = 16 * half; part < 16 * half + 16; part++)
+        cp_async16(s.raw + r * TA_WIN_LD + 16 * part, wr + 16 * part);
     }
   }
+  if (half == 0) s.row[r] = row;  // read after the barriers below
   cp_async_commit();  // the rows' group (empty when there are none)
   // the queries' copies (the first group) have landed; the rows may still be
   // in flight while the queries are converted
@@ -235,13 +234,7 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     }
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float M = __uint_as_float(mx << 16);
-    int e = 0;
-    if (M > 0.0f && M <= 3.3895314e38f) {  // finite, nonzero: 2^14 <= M 2^e < 2^15
-      int ex;
-      frexpf(M, &ex);
-      e = 15 - ex;
-    }
+    const int e = q_pow2_exponent(mx);
     const int e1 = e / 2, e2 = e - e1;  // each within a float's exponent range
     const float f = pow2i(e1), f2 = pow2i(e2);
     if (g == 0) {
@@ -265,10 +258,9 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
 
   // ---- dequantise into the fp16 tile: two threads per row, 256 channels each
   if (nk > 0) {
-    const int r = t & (TA_KEYS - 1), half = t >> 7;
     uint8_t* trow = s.tile + r * 128;
     const int sw = r & 7;
-    if (s.row[r] < 0) {
+    if (row < 0) {
 #pragma unroll 1
       for (int j = 0; j < 32; j++)
         *reinterpret_cast<uint4*>(trow + (4 * half + (j >> 3)) * TA_KB + (((j & 7) ^ sw) << 4)) =
@@ -413,29 +405,39 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     if (!done && ok && lane == 0) set_status(p.status, ST_TIMEOUT);
     live = __syncthreads_and(done);
   }
-  if (live) {
-    tc_fence_after();
+  cluster_wait_acquire();  // (the arrival above) every owner's barrier is ready
+  if (c < TA_SPARSE && t == 0) mbar_arrive_expect_tx(&s.rbar, TA_RECV_BYTES);
+  {
+    // every CTA sends all of its bytes (zeros, with weight 0, when it has
+    // no keys), so each owner's count is fixed
     const int chl = 32 * (warp & 3) + lane;
+    if (live) tc_fence_after();
 #pragma unroll 1
     for (int cb = 2 * (warp >> 2); cb < 2 * (warp >> 2) + 2; cb++) {
-      uint32_t o[16];
-      tmem_ld_x16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + TA_O_COL + 16 * cb, o);
-      tmem_ld_wait();
-      uint32_t hv[8];
+      uint32_t hv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (live) {
+        uint32_t o[16];
+        tmem_ld_x16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + TA_O_COL + 16 * cb, o);
+        tmem_ld_wait();
 #pragma unroll
-      for (int k = 0; k < 8; k++)
-        hv[k] = h2u(__floats2half2_rn(__uint_as_float(o[2 * k]) * s.linv[2 * k],
-                                      __uint_as_float(o[2 * k + 1]) * s.linv[2 * k + 1]));
-      uint4* dst = reinterpret_cast<uint4*>(
-          cluster.map_shared_rank(s.raw + TA_RECV_OFF + ((c * 128 + chl) * CSA2_H) * 2, cb));
-      dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        for (int k = 0; k < 8; k++)
+          hv[k] = h2u(__floats2half2_rn(__uint_as_float(o[2 * k]) * s.linv[2 * k],
+                                        __uint_as_float(o[2 * k + 1]) * s.linv[2 * k + 1]));
+      }
+      const uint32_t dst = mapa_rank(s.raw + TA_RECV_OFF + ((c * 128 + chl) * CSA2_H) * 2, cb);
+      const uint32_t bar = mapa_rank(&s.rbar, cb);
+      st_async_v4(dst, make_uint4(hv[0], hv[1], hv[2], hv[3]), bar);
+      st_async_v4(dst + 16, make_uint4(hv[4], hv[5], hv[6], hv[7]), bar);
     }
   }
-  if (t < CSA2_H) {
-    const float2 ml = live ? make_float2(s.m[t], s.lsum[t]) : make_float2(-INFINITY, 0.0f);
-#pragma unroll 1
-    for (int o2 = 0; o2 < TA_SPARSE; o2++) *cluster.map_shared_rank(&s.ml[c][t], o2) = ml;
+  if (t < CSA2_H / 2 * TA_SPARSE) {  // (max, sum) of heads 2j, 2j + 1 to owner o2
+    const int j = t & 7, o2 = t >> 3;
+    float4 v = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
+    if (live) v = make_float4(s.m[2 * j], s.lsum[2 * j], s.m[2 * j + 1], s.lsum[2 * j + 1]);
+    st_async_v4(mapa_rank(&s.ml[c][2 * j], o2),
+                make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                           __float_as_uint(v.w)),
+                mapa_rank(&s.rbar, o2));
   }
   tc_fence_before();
   __syncthreads();
@@ -443,10 +445,11 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     tc_fence_after();
     tmem_dealloc(tmem, TA_TMEM_COLS);
   }
-  cluster.sync();  // every partial has arrived; no remote access after this
 
   // ---- owners: log-sum-exp merge of the five partials of 128 channels
   if (c < TA_SPARSE) {
+    // every source's partial has landed here (bounded wait)
+    if (!mbar_wait_cluster(&s.rbar, 0) && t == 0) set_status(p.status, ST_TIMEOUT);
     if (t < CSA2_H) {
       float M = -INFINITY;
 #pragma unroll

@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergePa
   extern __shared__ __align__(16) uint8_t smem_raw[];
   CpMergeSmem& sm = *reinterpret_cast<CpMergeSmem*>(smem_raw);
   pdl_launch_dependents();
+  cluster_select_prologue(sm.sel, /*cluster_wide=*/false);
   pdl_wait();
   const int b = blockIdx.x, t = threadIdx.x;
   const int n = p.world * p.top_k;  // <= CPM_NT * CPM_KPT, checked by the host

@@ -71,6 +71,55 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// -------------------------------------------- cluster shared memory (DSMEM)
+// The shared::cluster address of rank's copy of a local shared variable.
+__device__ __forceinline__ uint32_t mapa_rank(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+// 16-byte store into another CTA's shared memory whose arrival is counted
+// (as 16 bytes of transaction) on the receiver's mbarrier; the sender does
+// not wait for it.
+__device__ __forceinline__ void st_async_v4(uint32_t dst, uint4 v, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(dst),
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
+      : "memory");
+}
+// Split cluster barrier: every thread of every CTA arrives (release), and
+// later waits (acquire).  Arrivals and waits alternate per thread.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Bounded wait for a phase of a local mbarrier that other CTAs of the
+// cluster complete (acquire at cluster scope: their stores are visible
+// after it).  Returns false after `budget` cycles.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  long long budget = kWaitCycles) {
+  auto try_once = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (try_once()) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (try_once()) return true;
+    if (clock64() - t0 > budget) return false;
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -245,6 +294,27 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------- fp16 query scaling
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+// Queries reach the fp16 tensor-core operands as Q' = Q * 2^e per head, e
+// chosen from the head's largest |q| (bf16 magnitude bits; 0x7F80 and above
+// is inf/NaN) so that max |Q'| lies in [2^14, 2^15): no overflow, and every
+// element keeps fp16's precision down to 2^-24 of 2^15.  e = 0 for an
+// all-zero or non-finite head.  Callers scale by 2^e1 * 2^e2 and undo it on
+// the logits with 2^-e1 and 2^-e2 (e1 = e / 2, e2 = e - e1), each factor
+// inside a float's exponent range.
+__device__ __forceinline__ int q_pow2_exponent(uint32_t maxbits) {
+  const float M = __uint_as_float(maxbits << 16);
+  int e = 0;
+  if (M > 0.0f && M <= 3.3895314e38f) {
+    int ex;
+    frexpf(M, &ex);  // M = m 2^ex, m in [0.5, 1)
+    e = 15 - ex;
+  }
+  return e;
 }
 
 // ------------------------------------------------------------ misc

@@ -494,6 +494,7 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RescoreSmem& s = *reinterpret_cast<RescoreSmem*>(smem_raw);
   pdl_launch_dependents();
+  cluster_select_prologue(s.sel);
   const int b = blockIdx.y;
   const RescoreJob job = p.job[blockIdx.z];
   uint32_t bq[8];
@@ -532,7 +533,8 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
   };
   __syncthreads();
   cluster_select_topk<RS_NT, RS_KPT>(s.sel, key, id_of, p.top_k,
-                                     job.idx + (int64_t)b * job.idx_stride, job.idx_count + b);
+                                     job.idx + (int64_t)b * job.idx_stride, job.idx_count + b,
+                                     true, p.status);
 }
 
 // --------------------------------------------- block Top-k (pool) select
@@ -546,6 +548,7 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SelectSmem<BS_NT, BS_KPT>& sm = *reinterpret_cast<SelectSmem<BS_NT, BS_KPT>*>(smem_raw);
   pdl_launch_dependents();
+  cluster_select_prologue(sm);
   pdl_wait();  // the block maxima come from the scan
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(BS_NT) block_select_kernel(
     for (int u = 0; u < 4; u++) key[4 * j + u] = (e0 + 4 * j + u < nblk) ? float_key(f[u]) : 0u;
   }
   cluster_select_topk<BS_NT, BS_KPT>(sm, key, [](int e) { return e; }, k_req,
-                                     sel + (int64_t)b * sel_stride, sel_count + b);
+                                     sel + (int64_t)b * sel_stride, sel_count + b, true, status);
 }
 
 // ------------------------------------------------------------ launchers

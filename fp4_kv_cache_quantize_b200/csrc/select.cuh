@@ -25,9 +25,14 @@
 // (instruction fetch, not arithmetic, bounds this kernel's latency), so all
 // rounds run the same rolled loop body.
 // Cluster exchanges push each CTA's counts into every rank's shared memory
-// before a cluster barrier (remote stores do not wait), so every read after
-// a barrier is local and every rank can work out every rank's share of the
-// result.  The placement needs no further exchange: each rank knows how many
+// with asynchronous stores (st.async) that count their bytes on the
+// receiver's mbarrier: a rank waits only until every rank's counts have
+// landed in its own shared memory, never on a cluster barrier, and every
+// rank can work out every rank's share of the result from local reads.
+// Round parities alternate two receive buffers and two mbarriers; a rank can
+// send round r + 2's counts only after it has received round r + 1's from
+// every rank, which each sent after reading its round r buffer, so a buffer
+// is never overwritten while it is read.  The placement needs no further exchange: each rank knows how many
 // selected elements precede it and how many of its keys equal to the
 // threshold it takes, and places its own with one block prefix scan.
 #pragma once
@@ -46,8 +51,8 @@ constexpr int SEL_MAX_RANKS = 16;
 template <int NT, int KPT>
 struct SelectSmem {
   static constexpr int NW = NT / 32;
-  uint32_t hist[SEL_NB];                         // this CTA's counts of the round
-  uint32_t xbuf[2][SEL_MAX_RANKS][SEL_NB];       // every rank's counts, by round parity
+  alignas(16) uint32_t hist[2][SEL_NB];          // this CTA's counts, by round parity
+  alignas(16) uint32_t xbuf[2][SEL_MAX_RANKS][SEL_NB];  // every rank's counts, by round parity
   uint32_t wred[NW][4];                          // round 0: per-warp max, min, count
   alignas(16) uint32_t cinfo[SEL_MAX_RANKS][4];  // round 0: per-rank max, min, count
   uint32_t above[SEL_MAX_RANKS];                 // per rank: keys above the bracket
@@ -55,8 +60,30 @@ struct SelectSmem {
   uint32_t verdict[4];
   uint32_t fin[4];                               // this rank's rule: T, keys == T taken, first output slot
   uint32_t wsum[32];
+  uint64_t xbar[2];  // every rank's counts of the round have arrived (by parity)
+  uint64_t cbar;     // every rank's round-0 figures have arrived
+  uint64_t pad_;
 };
 static_assert(sizeof(SelectSmem<256, 4>) % 16 == 0, "keeps what follows 16-byte aligned");
+
+// Every thread of every CTA calls this before the selection, before any
+// other use of sm, with the same cluster_wide as the selection; it starts a
+// cluster barrier that the selection completes, so a kernel issues it early
+// (before waiting for its inputs) and other work hides the barrier.  No
+// other cluster barrier may come between the two.
+template <int NT, int KPT>
+__device__ __forceinline__ void cluster_select_prologue(SelectSmem<NT, KPT>& sm,
+                                                        bool cluster_wide = true) {
+  const int t = threadIdx.x;
+  for (int i = t; i < 2 * SEL_NB; i += NT) sm.hist[i / SEL_NB][i % SEL_NB] = 0u;
+  if (t == 0) {
+    mbar_init(&sm.xbar[0], 1);
+    mbar_init(&sm.xbar[1], 1);
+    mbar_init(&sm.cbar, 1);
+    fence_mbar_init();
+  }
+  if (cluster_wide && cg::this_cluster().num_blocks() > 1) cluster_arrive_release();
+}
 
 // Exclusive block-wide prefix sum of v over threads in index order.
 template <int NT>
@@ -174,19 +201,22 @@ __device__ __forceinline__ int round_shift(uint32_t span, int bits) {
   return nbits > bits ? nbits - bits : 0;
 }
 
-// Every thread of every CTA of the cluster calls this with the same k_req.
+// Every thread of every CTA of the cluster calls this with the same k_req,
+// after cluster_select_prologue.
 // key[j] is element (rank*NT + t)*KPT + j's key (0 = not a candidate).
 // id_of(e) maps a cluster-wide element index to the id written to out.
 // Writes out[0..k) (k = min(k_req, candidates)) in ascending element order,
 // out[k..k_req) = -1 and *out_count = k (rank 0 writes the last two).
 // With cluster_wide = false the calling CTA selects on its own (rank 0 of a
-// one-CTA selection) even inside a larger cluster.
+// one-CTA selection) even inside a larger cluster.  A wait for another
+// rank's counts that gives up (after kWaitCycles) sets ST_TIMEOUT in
+// *status (when given) and the result is not defined.
 // cluster_select_emit: the same selection, handing each selected element to
 // emit(output slot, id) instead of writing an array; returns k.
 template <int NT, int KPT, class IdOf, class Emit>
 __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
                                         IdOf id_of, int k_req, Emit emit,
-                                        bool cluster_wide = true) {
+                                        bool cluster_wide = true, uint32_t* status = nullptr) {
   static_assert(NT >= 64 && NT % 32 == 0, "at least 64 threads");
   static_assert(KPT <= 15, "4-bit per-lane counters");
   static_assert(NT * KPT < 65536, "16-bit packed counts");
@@ -196,13 +226,17 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
   const unsigned rank = cluster_wide ? cluster.block_rank() : 0u;
   const unsigned ncta = cluster_wide ? cluster.num_blocks() : 1u;
   const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-  auto csync = [&]() {
-    if (ncta > 1) cluster.sync();
-    else __syncthreads();
+  bool failed = false;  // a wait gave up: later waits are skipped
+  auto wait_counts = [&](uint64_t* bar, uint32_t parity) {
+    if (!failed && !mbar_wait_cluster(bar, parity)) {
+      failed = true;
+      if (status) set_status(status, ST_TIMEOUT);
+    }
   };
+  // every rank's barriers are initialised (the prologue's arrival)
+  if (ncta > 1) cluster_wait_acquire();
 
   // ---- round 0: maximum, minimum and number of candidates
-  if (t < SEL_NB) sm.hist[t] = 0u;
   {
     uint32_t mx = 0u, mn = FULL, cnt = 0u;
 #pragma unroll
@@ -233,15 +267,18 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
       a = __reduce_max_sync(FULL, a);
       b = __reduce_min_sync(FULL, b);
       c = __reduce_add_sync(FULL, c);
-      if (lane < (int)ncta) {  // push this CTA's figures to every rank
-        uint32_t* dst = ncta > 1 ? cluster.map_shared_rank(&sm.cinfo[rank][0], lane)
-                                 : &sm.cinfo[0][0];
-        dst[0] = a;
-        dst[1] = b;
-        dst[2] = c;
+      if (ncta > 1) {  // push this CTA's figures to every rank
+        if (lane == 0) mbar_arrive_expect_tx(&sm.cbar, 16u * ncta);
+        __syncwarp();
+        if (lane < (int)ncta)
+          st_async_v4(mapa_rank(&sm.cinfo[rank][0], lane), make_uint4(a, b, c, 0u),
+                      mapa_rank(&sm.cbar, lane));
+      } else if (lane == 0) {
+        *reinterpret_cast<uint4*>(sm.cinfo[0]) = make_uint4(a, b, c, 0u);
       }
     }
-    csync();
+    if (ncta > 1) wait_counts(&sm.cbar, 0u);
+    else __syncthreads();
   }
   uint32_t gmx = 0u, gmn = FULL, gcnt = 0u, cnt_below = 0u;
 #pragma unroll
@@ -271,28 +308,35 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
     if (t < SEL_MAX_RANKS) sm.above[t] = 0u;
     int mode = 0;  // 1: the whole bin; 2: one key value
     uint32_t nlo = lo, nhi = hi;
+#pragma unroll 1  // one copy of the body: its instructions are fetched once
     for (int round = 0; round < 12; round++) {
       const uint32_t span = hi - lo;  // > 0 here
       const int par = round & 1;
       int s;
       if (round == 0) {
         s = round_shift(span, 4);
-        count16<KPT>(sm.hist, key, lo, span, s);
+        count16<KPT>(sm.hist[par], key, lo, span, s);
       } else {
         s = round_shift(span, 6);
-        count64<KPT>(sm.hist, key, lo, span, s);
+        count64<KPT>(sm.hist[par], key, lo, span, s);
       }
       __syncthreads();
-      if (t < SEL_NB) {  // push this CTA's counts to every rank
-        const uint32_t v = sm.hist[t];
-        sm.hist[t] = 0u;
-        if (ncta > 1) {
-          for (unsigned r = 0; r < ncta; r++) *cluster.map_shared_rank(&sm.xbuf[par][rank][t], r) = v;
-        } else {
-          sm.xbuf[par][0][t] = v;
+      // the other parity's counts were pushed last round, before that
+      // round's find: clear them for the next round
+      if (t < SEL_NB) sm.hist[par ^ 1][t] = 0u;
+      if (ncta > 1) {  // push this CTA's counts to every rank, 16 bytes per thread
+        if (t == 0) mbar_arrive_expect_tx(&sm.xbar[par], (uint32_t)(SEL_NB * 4) * ncta);
+        for (int i = t; i < (SEL_NB / 4) * (int)ncta; i += NT) {
+          const int g = i % (SEL_NB / 4), r = i / (SEL_NB / 4);
+          st_async_v4(mapa_rank(&sm.xbuf[par][rank][4 * g], r),
+                      *reinterpret_cast<const uint4*>(&sm.hist[par][4 * g]),
+                      mapa_rank(&sm.xbar[par], r));
         }
+        wait_counts(&sm.xbar[par], (uint32_t)(round >> 1) & 1u);
+      } else {
+        if (t < SEL_NB) sm.xbuf[par][0][t] = sm.hist[par][t];
+        __syncthreads();
       }
-      csync();
       if (wid == 0) find_bin(sm, sm.xbuf[par], ncta, krem);
       __syncthreads();
       const uint32_t jb = sm.verdict[0], above = sm.verdict[1], inbin = sm.verdict[2];
@@ -376,9 +420,9 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
 template <int NT, int KPT, class IdOf>
 __device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
                                     IdOf id_of, int k_req, int32_t* out, int32_t* out_count,
-                                    bool cluster_wide = true) {
+                                    bool cluster_wide = true, uint32_t* status = nullptr) {
   const uint32_t k = cluster_select_emit(
-      sm, key, id_of, k_req, [out](int pos, int id) { out[pos] = id; }, cluster_wide);
+      sm, key, id_of, k_req, [out](int pos, int id) { out[pos] = id; }, cluster_wide, status);
   const unsigned rank = cluster_wide ? cg::this_cluster().block_rank() : 0u;
   if (rank == 0) {
     for (int i = (int)k + (int)threadIdx.x; i < k_req; i += NT) out[i] = -1;

@@ -114,6 +114,22 @@ def test_cp_paged_without_pool(lib, orc, world):
     check(lib, orc, wl, world, paged=True)
 
 
+def test_cp_query_magnitudes(lib, orc):
+    """Shards attend with the split-KV kernel: main queries whose heads span
+    bf16's range (1e-6 to 1e5, beyond fp16's 65,504, and all-zero heads)
+    must match the oracle with no overflow and no loss of small queries."""
+    wl = synth.make("cp", seed=540, B=2, n_rows=[6000, 900],
+                    modes=[FULL, REUSE, REINDEX], pool_blocks=2048, swa_len=[128, 60])
+    q = synth.bf16_bits_to_f32(wl.q).astype(np.float64)
+    scale = np.array([1e-6, 3e-5, 1e-3, 0.25, 1.0, 7.0, 100.0, 2e3,
+                      3e4, 6.5e4, 1e5, 1e5, 0.0, 1.0, 1e-6, 5e4])
+    for l in range(wl.L):
+        q[l] *= np.roll(scale, 3 * l)[None, :, None]
+    wl.q = synth.to_bf16_bits(q.astype(np.float32))
+    assert np.abs(synth.bf16_bits_to_f32(wl.q)).max() > 65504.0
+    check(lib, orc, wl, 2, paged=False)
+
+
 def test_cp_attention_only_window(lib, orc):
     """A sequence with no global entries: every shard's rows are empty and
     the output is the window-only attention of the rank holding the window."""
