@@ -1010,58 +1010,82 @@ def run_gpu(args, wl, rank, world):
     # Steps run back to back with the copies overlapped: the host->device
     # copy of step i+1's inputs and the device->host copy of step i-1's
     # results run on their own streams while step i computes (two sets of
-    # device input and output buffers).  No L2 flush here: every step streams
-    # 134 MB of indexer K, more than the 126 MB L2.
+    # device input and output buffers).  E2E_UNROLL consecutive steps (their
+    # copies and their csa2_layer_group calls, on three streams with the
+    # dependencies above) are captured as one CUDA graph, so the host issues
+    # one launch per E2E_UNROLL steps and its own speed does not set the
+    # step time.  No L2 flush here: every step streams 134 MB of indexer K,
+    # more than the 126 MB L2.
     sets = [(q_idx, w_h, q, grp)]
     q_idx2, w_h2, q2 = torch.empty_like(q_idx), torch.empty_like(w_h), torch.empty_like(q)
     grp2 = csa2.LayerGroup(kv, wl.modes, q_idx2, w_h2, q2, swa, swa_len, top_k=wl.top_k,
                            pool_blocks=wl.pool_blocks)
     sets.append((q_idx2, w_h2, q2, grp2))
-    if step_launch == "cuda_graph":
-        csa2.csa2_layer_group(grp2, ws)   # set up outside the capture
-        torch.cuda.synchronize()
-        g2 = capture(grp2)
-        runs = [graph.replay, g2.replay if isinstance(g2, torch.cuda.CUDAGraph) else (
-            lambda: csa2.csa2_layer_group(grp2, ws))]
-    else:
-        runs = [step, lambda: csa2.csa2_layer_group(grp2, ws)]
+    csa2.csa2_layer_group(grp2, ws)   # set up outside the capture
+    torch.cuda.synchronize()
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     h_outs = [h_out, torch.empty_like(h_out).pin_memory()]
     h_idxs = [h_idx, torch.empty_like(h_idx).pin_memory()]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    for e in ev_done + ev_out:
-        e.record(stream)
+
+    def e2e_steps(n):
+        """n steps with overlapped copies, issued on the current stream."""
+        main = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(main)
+        ev_done = [fork, fork]
+        ev_out = [fork, fork]
+        for i in range(n):
+            j = i % 2
+            d_qi, d_w, d_q, g = sets[j]
+            ev_in = torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_done[j])          # step i-2 no longer reads set j
+                d_qi.copy_(h_q_idx, non_blocking=True)
+                d_w.copy_(h_w, non_blocking=True)
+                d_q.copy_(h_q, non_blocking=True)
+                ev_in.record(s_in)
+            main.wait_event(ev_in)
+            main.wait_event(ev_out[j])               # step i-2's results have left set j
+            csa2.csa2_layer_group(g, ws)
+            ev_done[j] = torch.cuda.Event()
+            ev_done[j].record(main)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[j])
+                h_outs[j].copy_(g.out, non_blocking=True)
+                h_idxs[j].copy_(g.idx, non_blocking=True)
+                ev_out[j] = torch.cuda.Event()
+                ev_out[j].record(s_out)
+        main.wait_event(ev_out[0])
+        main.wait_event(ev_out[1])
+
+    E2E_UNROLL = 10
+    reps = max(1, K // E2E_UNROLL)
+    e2e_graph = None
+    if step_launch == "cuda_graph":
+        try:
+            e2e_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(e2e_graph):
+                e2e_steps(E2E_UNROLL)
+            torch.cuda.synchronize()
+        except Exception:  # noqa: BLE001  (direct launches below)
+            torch.cuda.synchronize()
+            e2e_graph = None
+    e2e_launch = f"cuda_graph of {E2E_UNROLL} steps" if e2e_graph else "direct"
+    for _ in range(2):  # warm-up
+        e2e_graph.replay() if e2e_graph else e2e_steps(E2E_UNROLL)
     t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier()
-    t0e.record(s_in)
-    for i in range(K):
-        j = i % 2
-        d_qi, d_w, d_q, g = sets[j]
-        with torch.cuda.stream(s_in):
-            s_in.wait_event(ev_done[j])          # step i-2 no longer reads set j
-            d_qi.copy_(h_q_idx, non_blocking=True)
-            d_w.copy_(h_w, non_blocking=True)
-            d_q.copy_(h_q, non_blocking=True)
-            ev_in[j].record(s_in)
-        stream.wait_event(ev_in[j])
-        stream.wait_event(ev_out[j])             # step i-2's results have left set j
-        runs[j]()
-        ev_done[j].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_done[j])
-            h_outs[j].copy_(g.out, non_blocking=True)
-            h_idxs[j].copy_(g.idx, non_blocking=True)
-            ev_out[j].record(s_out)
-    s_out.wait_event(ev_done[(K - 1) % 2])
-    t1e.record(s_out)
+    t0e.record(stream)
+    for _ in range(reps):
+        e2e_graph.replay() if e2e_graph else e2e_steps(E2E_UNROLL)
+    t1e.record(stream)
     torch.cuda.synchronize()
     barrier()
     csa2.csa2_sync_status(ws)
-    t_e2e = max_over_ranks(t0e.elapsed_time(t1e) / K, dist, dev)
-    assert torch.equal(h_idxs[(K - 1) % 2], grp.idx.cpu())
+    K_e2e = reps * E2E_UNROLL
+    t_e2e = max_over_ranks(t0e.elapsed_time(t1e) / K_e2e, dist, dev)
+    assert torch.equal(h_idxs[0], grp.idx.cpu()) and torch.equal(h_idxs[1], grp.idx.cpu())
 
     with_cpu = rank == 0 and world == 1 and not args.no_cpu
     append = time_cache_append(csa2, wl, dev, stream, K, args.warmup, with_cpu)
@@ -1135,11 +1159,14 @@ def run_gpu(args, wl, rank, world):
             "e2e": {"value": job_throughput(units, world, t_e2e), "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": t_e2e,
-                    "timing": (f"{K} back-to-back steps through the C ABI; each step's inputs "
+                    "launch": e2e_launch,
+                    "timing": (f"{K_e2e} back-to-back steps through the C ABI; each step's inputs "
                                "copied from pinned host memory and its outputs (attention "
                                "output, indices) copied back, on separate streams overlapping "
-                               "the neighbouring steps' compute; no L2 flush (134 MB of "
-                               "indexer K per step exceeds the 126 MB L2)")},
+                               "the neighbouring steps' compute; every "
+                               f"{E2E_UNROLL} steps' copies and calls replayed as one CUDA "
+                               "graph; no L2 flush (134 MB of indexer K per step exceeds the "
+                               "126 MB L2)")},
             "back_to_back": b2b,
             "configs": others,
             "layer_sequential": seq,

@@ -42,19 +42,13 @@ namespace csa2 {
 
 namespace cg = cooperative_groups;
 
-constexpr int TA_NT = 256;
+constexpr int TA_NT = 512;
+constexpr int TA_TPR = TA_NT / 128;  // threads per key row (4): a quarter of the row each
 constexpr int TA_KEYS = 128;                        // keys per CTA: the MMA's M
 constexpr int TA_SPARSE = CSA2_MAX_TOPK / TA_KEYS;  // CTAs of the sparse branch
 constexpr int TA_CTAS = TA_SPARSE + 1;              // and the window's
 static_assert(CSA2_W == TA_KEYS, "one CTA holds the whole window");
 constexpr int TA_KB = TA_KEYS * 128;                // one 64-channel block of the tile
-constexpr int TA_CODE_LD = 272;                     // padded shared-memory row strides
-constexpr int TA_SCALE_LD = 48;
-constexpr int TA_WIN_LD = 528;
-constexpr int TA_SCALE_OFF = TA_KEYS * TA_CODE_LD;
-constexpr int TA_RECV_OFF = TA_SCALE_OFF + TA_KEYS * TA_SCALE_LD;
-constexpr int TA_RAW_BYTES = TA_KEYS * TA_WIN_LD;
-static_assert(TA_RECV_OFF + TA_CTAS * 128 * CSA2_H * 2 <= TA_RAW_BYTES, "receive buffer");
 constexpr uint32_t TA_IDESC_QK = idesc_f16_f32(128, 16, false);
 constexpr uint32_t TA_IDESC_PV = idesc_f16_f32(128, 16, true);
 constexpr uint32_t TA_TMEM_COLS = 128;  // S^T in columns [0, 16), O^T in [64, 128)
@@ -67,10 +61,10 @@ struct TaSmem {
   alignas(1024) uint8_t tile[8 * TA_KB];
   alignas(1024) uint8_t q[8 * 2048];       // Q': channel block kb, 16 rows (heads) of 128 B
   alignas(1024) uint8_t p[2 * 2048];       // P^T: key block kb, 16 rows (heads) of 128 B
-  // gathered rows: the window's E4M3 rows, or FP4 codes | scales | the
-  // normalised partials this CTA receives as the owner of a channel block;
-  // after the dequantisation its first 8 KB hold the logits [head][key]
-  alignas(16) uint8_t raw[TA_RAW_BYTES];
+  alignas(16) float sS[CSA2_H * TA_KEYS];  // logits [head][key], log2 units
+  // the normalised partials this CTA receives as the owner of a channel
+  // block: [source CTA][channel][head] fp16
+  alignas(16) uint8_t recv[TA_CTAS * 128 * CSA2_H * 2];
   int64_t row[TA_KEYS];
   float scl1[CSA2_H], scl2[CSA2_H];        // logit = acc * scl1 * scl2 (log2 units)
   float m[CSA2_H], lsum[CSA2_H], linv[CSA2_H];
@@ -149,11 +143,13 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
 
   // ---- this CTA's keys.  b runs over sequences x queries: query tq of
   // sequence bp sees the sequence's entries minus the drafts after it, and
-  // the window rows that end at its own entry.  Threads r and r + 128 both
-  // resolve key r's row (from the same index) and copy half of it each, so
-  // no thread waits for another before its copies start.
+  // the window rows that end at its own entry.  Threads r, r + 128, r + 256
+  // and r + 384 all resolve key r's row (from the same index) and copy a
+  // quarter of it each, so no thread waits for another before its copies
+  // start.
   const int bp = b / p.nq, tq = b - bp * p.nq, later = p.nq - 1 - tq;
-  const int r = t & (TA_KEYS - 1), half = t >> 7;
+  const int r = t & (TA_KEYS - 1), qq = t >> 7;
+  static_assert(TA_TPR == 4, "four threads per key row");
   const int32_t* idx = L.idx + (int64_t)b * p.idx_stride;
   const int kt = c * TA_KEYS + r;
   // this thread's index, read before the counts arrive (within the index
@@ -167,6 +163,12 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   C = C - later < 0 ? 0 : C - later;
   int nk;          // candidate keys of this CTA: keys j < nk
   int64_t row = -1;  // key r's row of the cache (or of the window), -1: none
+  // this thread's quarter of row r, loaded straight into registers (no
+  // shared-memory staging): the dequantisation below consumes it
+  uint4 rv[8];
+  uint2 sv = make_uint2(0u, 0u);
+#pragma unroll
+  for (int i = 0; i < 8; i++) rv[i] = make_uint4(0u, 0u, 0u, 0u);
   if (!window) {
     int n_idx = L.idx_count[b];
     if (n_idx < 0 || n_idx > p.idx_stride) {
@@ -174,25 +176,19 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
       n_idx = n_idx < 0 ? 0 : p.idx_stride;
     }
     nk = min(max(n_idx - c * TA_KEYS, 0), TA_KEYS);
-    if (L.idx_copy && half == 0) {  // Reuse layer: publish the indices it used
+    if (L.idx_copy && qq == 0) {  // Reuse layer: publish the indices it used
       if (kt < p.idx_stride) L.idx_copy[(int64_t)b * p.idx_stride + kt] = pos_t;
       if (c == 0 && t == 0) L.idx_copy_count[b] = L.idx_count[b];
     }
     if (r < nk) {
       if (pos_t >= 0 && pos_t < C) row = ta_kv_row(p, bp, pos_t);
-      if (row < 0 && half == 0) set_status(p.status, ST_DEVICE_CHECK);
+      if (row < 0 && qq == 0) set_status(p.status, ST_DEVICE_CHECK);
     }
-    if (row >= 0) {  // 16 code chunks and 2 scale chunks: 9 per thread
-      const uint8_t* cg_ = p.codes + row * (CSA2_D / 2);
-      const uint8_t* sg_ = p.scales + row * (CSA2_D / 16);
-#pragma unroll 1
-      for (int part = 9 * half; part < 9 * half + 9; part++) {
-        if (part < 16)
-          cp_async16(s.raw + r * TA_CODE_LD + 16 * part, cg_ + 16 * part);
-        else
-          cp_async16(s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * (part - 16),
-                     sg_ + 16 * (part - 16));
-      }
+    if (row >= 0) {  // channels [128 qq, 128 qq + 128): 64 code bytes, 8 scales
+      const uint4* cg_ = reinterpret_cast<const uint4*>(p.codes + row * (CSA2_D / 2) + 64 * qq);
+#pragma unroll
+      for (int i = 0; i < 4; i++) rv[i] = __ldg(cg_ + i);
+      sv = __ldg(reinterpret_cast<const uint2*>(p.scales + row * (CSA2_D / 16) + 8 * qq));
     }
   } else {
     int n_win = p.swa_len[bp];
@@ -203,37 +199,35 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     const int win_end = n_win - later < 0 ? 0 : n_win - later;
     const int win_lo = win_end > CSA2_W ? win_end - CSA2_W : 0;
     nk = win_end - win_lo;
-    if (r < nk) {  // 32 chunks of 16 E4M3 values: 16 per thread
+    if (r < nk) {  // channels [128 qq, 128 qq + 128): 128 E4M3 values
       row = r;
-      const uint8_t* wr = L.swa + ((int64_t)bp * p.swa_rows + win_lo + r) * CSA2_D;
-#pragma unroll 1
-      for (int part = 16 * half; part < 16 * half + 16; part++)
-        cp_async16(s.raw + r * TA_WIN_LD + 16 * part, wr + 16 * part);
+      const uint4* wr = reinterpret_cast<const uint4*>(
+          L.swa + ((int64_t)bp * p.swa_rows + win_lo + r) * CSA2_D + 128 * qq);
+#pragma unroll
+      for (int i = 0; i < 8; i++) rv[i] = __ldg(wr + i);
     }
   }
-  if (half == 0) s.row[r] = row;  // read after the barriers below
-  cp_async_commit();  // the rows' group (empty when there are none)
-  // the queries' copies (the first group) have landed; the rows may still be
-  // in flight while the queries are converted
-  asm volatile("cp.async.wait_group %0;" ::"n"(1) : "memory");
+  if (qq == 0) s.row[r] = row;  // read after the barriers below
+  // the queries' copies have landed; the rows may still be in flight (in
+  // registers) while the queries are converted
+  cp_async_wait_all();
   __syncthreads();
 
-  // ---- Q' = Q * 2^e_h in fp16, max |Q'_h| in [2^14, 2^15): 16 threads per
-  // head, 32 channels each
+  // ---- Q' = Q * 2^e_h in fp16, max |Q'_h| in [2^14, 2^15): warp h converts
+  // head h, 16 channels per lane
   {
-    const int h = t >> 4, g = t & 15;
-    const uint4* src = reinterpret_cast<const uint4*>(s.tile + h * (CSA2_D * 2) + g * 64);
-    uint4 v[4];
+    const int h = warp, g = lane;
+    const uint4* src = reinterpret_cast<const uint4*>(s.tile + h * (CSA2_D * 2) + g * 32);
+    uint4 v[2];
     uint32_t mx = 0u;
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
+    for (int k = 0; k < 2; k++) {
       v[k] = src[k];
       const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
       for (int j = 0; j < 4; j++) mx = max(mx, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
     }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mx = __reduce_max_sync(0xffffffffu, mx);
     const int e = q_pow2_exponent(mx);
     const int e1 = e / 2, e2 = e - e1;  // each within a float's exponent range
     const float f = pow2i(e1), f2 = pow2i(e2);
@@ -242,40 +236,38 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
       s.scl2[h] = p.scale_log2 * pow2i(-e2);
     }
 #pragma unroll
-    for (int k = 0; k < 4; k++) {  // channels 32 g + 8 k .. + 8: block g / 2, chunk 4 (g & 1) + k
+    for (int k = 0; k < 2; k++) {  // channels 16 g + 8 k .. + 8: block g / 4, chunk 2 (g & 3) + k
       const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
       uint32_t o4[4];
 #pragma unroll
       for (int j = 0; j < 4; j++)
         o4[j] = h2u(__floats2half2_rn(__uint_as_float(w[j] << 16) * f * f2,
                                       __uint_as_float(w[j] & 0xFFFF0000u) * f * f2));
-      *reinterpret_cast<uint4*>(s.q + (g >> 1) * 2048 + sw_off(h, 4 * (g & 1) + k)) =
+      *reinterpret_cast<uint4*>(s.q + (g >> 2) * 2048 + sw_off(h, 2 * (g & 3) + k)) =
           make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
   }
-  cp_async_wait_all();
-  __syncthreads();  // the rows have landed; the raw queries in the tile are consumed
+  __syncthreads();  // the raw queries in the tile are consumed
 
-  // ---- dequantise into the fp16 tile: two threads per row, 256 channels each
+  // ---- dequantise into the fp16 tile: four threads per row, 128 channels
+  // (channel blocks 2 qq and 2 qq + 1) each
   if (nk > 0) {
     uint8_t* trow = s.tile + r * 128;
     const int sw = r & 7;
     if (row < 0) {
 #pragma unroll 1
-      for (int j = 0; j < 32; j++)
-        *reinterpret_cast<uint4*>(trow + (4 * half + (j >> 3)) * TA_KB + (((j & 7) ^ sw) << 4)) =
+      for (int j = 0; j < 16; j++)
+        *reinterpret_cast<uint4*>(trow + (2 * qq + (j >> 3)) * TA_KB + (((j & 7) ^ sw) << 4)) =
             make_uint4(0, 0, 0, 0);
     } else if (!window) {
-      const uint8_t* cr = s.raw + r * TA_CODE_LD + 128 * half;
-      const uint8_t* sr = s.raw + TA_SCALE_OFF + r * TA_SCALE_LD + 16 * half;
-#pragma unroll 1
-      for (int i = 0; i < 8; i++) {  // 16 code bytes: channels 256 half + 32 i + [0, 32)
-        const uint4 cv = *reinterpret_cast<const uint4*>(cr + 16 * i);
+#pragma unroll
+      for (int i = 0; i < 4; i++) {  // 16 code bytes: channels 128 qq + 32 i + [0, 32)
+        const uint4 cv = rv[i];
         const uint32_t words[4] = {cv.x, cv.y, cv.z, cv.w};
-        const uint32_t sb = *reinterpret_cast<const uint16_t*>(sr + 2 * i);  // groups 2i, 2i+1
+        const uint32_t sb = ((i < 2 ? sv.x : sv.y) >> (16 * (i & 1))) & 0xFFFFu;  // groups 2i, 2i+1
         const __half s0 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sb & 0xFF), __NV_E4M3));
         const __half s1 = __half(__nv_cvt_fp8_to_halfraw((uint8_t)(sb >> 8), __NV_E4M3));
-        uint8_t* dst = trow + (4 * half + (i >> 1)) * TA_KB;
+        uint8_t* dst = trow + (2 * qq + (i >> 1)) * TA_KB;
 #pragma unroll
         for (int q4 = 0; q4 < 4; q4++) {  // 8 channels per 16-byte store
           const uint32_t word = words[q4];
@@ -291,10 +283,9 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
         }
       }
     } else {
-      const uint8_t* wr = s.raw + r * TA_WIN_LD + 256 * half;
-#pragma unroll 1
-      for (int j = 0; j < 16; j++) {  // 16 E4M3 bytes: channels 256 half + 16 j + [0, 16)
-        const uint4 v = *reinterpret_cast<const uint4*>(wr + 16 * j);
+#pragma unroll
+      for (int j = 0; j < 8; j++) {  // 16 E4M3 bytes: channels 128 qq + 16 j + [0, 16)
+        const uint4 v = rv[j];
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
         uint32_t hv[8];
 #pragma unroll
@@ -304,7 +295,7 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
           hv[2 * k + 1] = h2u(__half2(__nv_cvt_fp8x2_to_halfraw2(
               (__nv_fp8x2_storage_t)(wv[k] >> 16), __NV_E4M3)));
         }
-        uint8_t* dst = trow + (4 * half + (j >> 2)) * TA_KB;
+        uint8_t* dst = trow + (2 * qq + (j >> 2)) * TA_KB;
         const int cc = 2 * (j & 3);
         *reinterpret_cast<uint4*>(dst + ((cc ^ sw) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ sw) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
@@ -324,53 +315,51 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
 #pragma unroll 1
     for (int i = 0; i < 32; i++) {  // K = 512 in 32 steps: block kb = i / 4, 32-byte step i % 4
       const uint32_t kb = (uint32_t)i >> 2, sub = (uint32_t)i & 3;
-      umma_bf16(tmem, da + ((kb * TA_KB + 32 * sub) >> 4), db + ((kb * 2048 + 32 * sub) >> 4),
-                TA_IDESC_QK, i != 0);
+      umma_bf16(tmem + 16 * sub, da + ((kb * TA_KB + 32 * sub) >> 4), db + ((kb * 2048 + 32 * sub) >> 4),
+                TA_IDESC_QK, kb != 0);
     }
     umma_commit(&s.mbar);
   }
-  float* sS = reinterpret_cast<float*>(s.raw);  // logits [head][key], log2 units
+  float* sS = s.sS;
   bool ok = true;
   if (nk > 0 && warp < 4) {
     ok = __all_sync(0xffffffffu, mbar_wait(&s.mbar, 0, nullptr));
     if (!ok && lane == 0) set_status(p.status, ST_TIMEOUT);
     tc_fence_after();
-    uint32_t r[16];
-    tmem_ld_x16(tmem + ((uint32_t)(32 * warp) << 16), r);
+    uint32_t r[4][16];
+#pragma unroll
+    for (int a = 0; a < 4; a++) tmem_ld_x16(tmem + ((uint32_t)(32 * warp) << 16) + 16 * a, r[a]);
     tmem_ld_wait();
     const int key = 32 * warp + lane;
     const bool valid = ok && key < nk && s.row[key] >= 0;
 #pragma unroll
-    for (int h = 0; h < 16; h++)
-      sS[h * TA_KEYS + key] = valid ? __uint_as_float(r[h]) * s.scl1[h] * s.scl2[h] : -INFINITY;
+    for (int h = 0; h < 16; h++) {
+      const float acc = (__uint_as_float(r[0][h]) + __uint_as_float(r[1][h])) +
+                        (__uint_as_float(r[2][h]) + __uint_as_float(r[3][h]));
+      sS[h * TA_KEYS + key] = valid ? acc * s.scl1[h] * s.scl2[h] : -INFINITY;
+    }
   }
   __syncthreads();
-  // ---- softmax: 16 threads per head, 8 keys each; P^T in fp16, the sum
+  // ---- softmax: warp h for head h, 4 keys per lane; P^T in fp16, the sum
   // of the fp16 probabilities the MMA reads
   if (nk > 0) {
-    const int h = t >> 4, g = t & 15;
-    const float4* src = reinterpret_cast<const float4*>(sS + h * TA_KEYS + 8 * g);
-    const float4 x0 = src[0], x1 = src[1];
-    float m = fmaxf(fmaxf(fmaxf(x0.x, x0.y), fmaxf(x0.z, x0.w)),
-                    fmaxf(fmaxf(x1.x, x1.y), fmaxf(x1.z, x1.w)));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    uint32_t pv[4];
-    float l = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const __half2 ph = m == -INFINITY ? __floats2half2_rn(0.0f, 0.0f)
-                                        : __floats2half2_rn(exp2f(xs[2 * k] - m),
-                                                            exp2f(xs[2 * k + 1] - m));
-      const float2 pf = __half22float2(ph);
-      l += pf.x + pf.y;
-      pv[k] = h2u(ph);
+    const int h = warp, g = lane;
+    const float4 x = *reinterpret_cast<const float4*>(sS + h * TA_KEYS + 4 * g);
+    const float m = warp_max_f32(fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+    __half2 ph0, ph1;
+    if (m == -INFINITY) {
+      ph0 = ph1 = __floats2half2_rn(0.0f, 0.0f);
+    } else {
+      ph0 = __floats2half2_rn(exp2f(x.x - m), exp2f(x.y - m));
+      ph1 = __floats2half2_rn(exp2f(x.z - m), exp2f(x.w - m));
     }
-    *reinterpret_cast<uint4*>(s.p + (g >> 3) * 2048 + sw_off(h, g & 7)) =
-        make_uint4(pv[0], pv[1], pv[2], pv[3]);
+    const float2 p0 = __half22float2(ph0), p1 = __half22float2(ph1);
+    float l = (p0.x + p0.y) + (p1.x + p1.y);
+    // keys 4g .. 4g + 3: key block g / 16, 16-byte chunk (g / 2) % 8, half g % 2
+    *reinterpret_cast<uint2*>(s.p + (g >> 4) * 2048 + sw_off(h, (g >> 1) & 7) + 8 * (g & 1)) =
+        make_uint2(h2u(ph0), h2u(ph1));
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     if (g == 0) {
       s.m[h] = m;
       s.lsum[h] = l;
@@ -389,8 +378,8 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     tc_fence_after();
     const uint64_t da = sdesc_mn128(smem_u32(s.tile), TA_KB, 1024), db = sdesc_k128(smem_u32(s.p));
 #pragma unroll 1
-    for (int i = 0; i < 32; i++) {  // channel block cb = i / 8, 16 keys ks = i % 8
-      const uint32_t cb = (uint32_t)i >> 3, ks = (uint32_t)i & 7;
+    for (int i = 0; i < 32; i++) {  // 16 keys ks = i / 4, channel block cb = i % 4
+      const uint32_t cb = (uint32_t)i & 3, ks = (uint32_t)i >> 2;
       umma_bf16(tmem + TA_O_COL + 16 * cb, da + ((cb * 2 * TA_KB + ks * 2048) >> 4),
                 db + (((ks >> 2) * 2048 + (ks & 3) * 32) >> 4), TA_IDESC_PV, ks > 0);
     }
@@ -398,7 +387,7 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
   }
 
   // ---- normalised partial O^T -> the owners of the channel blocks: warp w
-  // reads TMEM lanes 32 (w % 4).., channel blocks 2 (w / 4) and 2 (w / 4) + 1
+  // reads TMEM lanes 32 (w % 4).., channel block w / 4
   bool live = nk > 0 && ok;
   if (nk > 0) {
     const bool done = __all_sync(0xffffffffu, ok && mbar_wait(&s.mbar, 1, nullptr));
@@ -412,8 +401,8 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
     // no keys), so each owner's count is fixed
     const int chl = 32 * (warp & 3) + lane;
     if (live) tc_fence_after();
-#pragma unroll 1
-    for (int cb = 2 * (warp >> 2); cb < 2 * (warp >> 2) + 2; cb++) {
+    {
+      const int cb = warp >> 2;
       uint32_t hv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
       if (live) {
         uint32_t o[16];
@@ -424,7 +413,7 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
           hv[k] = h2u(__floats2half2_rn(__uint_as_float(o[2 * k]) * s.linv[2 * k],
                                         __uint_as_float(o[2 * k + 1]) * s.linv[2 * k + 1]));
       }
-      const uint32_t dst = mapa_rank(s.raw + TA_RECV_OFF + ((c * 128 + chl) * CSA2_H) * 2, cb);
+      const uint32_t dst = mapa_rank(s.recv + ((c * 128 + chl) * CSA2_H) * 2, cb);
       const uint32_t bar = mapa_rank(&s.rbar, cb);
       st_async_v4(dst, make_uint4(hv[0], hv[1], hv[2], hv[3]), bar);
       st_async_v4(dst + 16, make_uint4(hv[4], hv[5], hv[6], hv[7]), bar);
@@ -466,32 +455,26 @@ __global__ void __launch_bounds__(TA_NT, 1) attn_tc_kernel(const AttnParams p) {
       for (int src = 0; src < TA_CTAS; src++) s.wts[src][t] = wv[src] * inv;
     }
     __syncthreads();
-    // two threads per channel, eight heads each
-    const int ch = t & 127, hh = 8 * (t >> 7);
-    float acc[8];
-#pragma unroll
-    for (int k = 0; k < 8; k++) acc[k] = 0.0f;
+    // four threads per channel, four heads each
+    const int ch = t & 127, hh = 4 * (t >> 7);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
     for (int src = 0; src < TA_CTAS; src++) {
-      const float4 w0 = *reinterpret_cast<const float4*>(&s.wts[src][hh]);
-      const float4 w1 = *reinterpret_cast<const float4*>(&s.wts[src][hh + 4]);
-      if (w0.x == 0.0f && w0.y == 0.0f && w0.z == 0.0f && w0.w == 0.0f && w1.x == 0.0f &&
-          w1.y == 0.0f && w1.z == 0.0f && w1.w == 0.0f)
-        continue;  // nothing from this source for these heads (its buffer may be stale)
-      const uint4 v = *reinterpret_cast<const uint4*>(s.raw + TA_RECV_OFF +
+      const float4 w4 = *reinterpret_cast<const float4*>(&s.wts[src][hh]);
+      if (w4.x == 0.0f && w4.y == 0.0f && w4.z == 0.0f && w4.w == 0.0f)
+        continue;  // nothing from this source for these heads
+      const uint2 v = *reinterpret_cast<const uint2*>(s.recv +
                                                       ((src * 128 + ch) * CSA2_H + hh) * 2);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      const float wt[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-      for (int k = 0; k < 4; k++) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-        acc[2 * k] = fmaf(wt[2 * k], f.x, acc[2 * k]);
-        acc[2 * k + 1] = fmaf(wt[2 * k + 1], f.y, acc[2 * k + 1]);
-      }
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+      acc[0] = fmaf(w4.x, f0.x, acc[0]);
+      acc[1] = fmaf(w4.y, f0.y, acc[1]);
+      acc[2] = fmaf(w4.z, f1.x, acc[2]);
+      acc[3] = fmaf(w4.w, f1.y, acc[3]);
     }
     uint16_t* out = L.out + ((int64_t)b * CSA2_H + hh) * CSA2_D + c * 128 + ch;
 #pragma unroll
-    for (int k = 0; k < 8; k++) {
+    for (int k = 0; k < 4; k++) {
       const __nv_bfloat16 v = __float2bfloat16_rn(acc[k]);
       out[k * CSA2_D] = *reinterpret_cast<const uint16_t*>(&v);
     }

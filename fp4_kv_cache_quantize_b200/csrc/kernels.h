@@ -56,11 +56,11 @@ struct ScanParams {
   int32_t nq_pass;   // 1..8
   int32_t tail;      // nq - (q_first + nq_pass): later queries not in this launch
   uint32_t* status;
-  uint32_t* sched;   // [2] tile counter and finished-CTA counter, zero at launch (workspace header)
+  uint32_t* sched;   // tile counter, zero at launch and again at exit (workspace header)
 };
 constexpr int SC_TILE = 128;
-// Word of the workspace header where the scan's two scheduling counters live
-// (the status word is word 0); both are zero between launches.
+// Word of the workspace header where the scan's tile counter lives (the
+// status word is word 0); it is zero between launches.
 constexpr int CSA2_WS_SCHED_WORD = 16;
 constexpr int CSA2_SCAN_QUERIES = 8;  // queries one scan launch scores (MMA N <= 64)
 

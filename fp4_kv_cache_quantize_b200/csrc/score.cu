@@ -156,12 +156,23 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
       // Tiles are handed out by a counter in the workspace header, one at a
       // time, so that CTAs that run faster take more of them (a fixed
       // interleave leaves a tail of slow CTAs); the next tile is requested
-      // while the current one is issued.
-      uint32_t next = atomicAdd(p.sched, 1u);
+      // while the current one is issued.  Every CTA stops at its first
+      // request past the last tile, so a launch makes exactly total +
+      // gridDim requests: the one that receives the last number is the last
+      // request of the launch, and it returns the counter to zero for the
+      // next launch (no end-of-kernel counter that every CTA would contend
+      // for).
+      const uint64_t last_req = (uint64_t)total + gridDim.x - 1u;
+      auto request = [&]() {
+        const uint32_t v = atomicAdd(p.sched, 1u);
+        if ((uint64_t)v == last_req) *p.sched = 0u;
+        return v;
+      };
+      uint32_t next = request();
       while (true) {
         const int64_t g = next;
         if (g >= total) break;
-        next = atomicAdd(p.sched, 1u);
+        next = request();
         const int b = (int)(g / p.tiles_per_seq), t = (int)(g % p.tiles_per_seq);
         if (b != cur_b) {
           C = visible_rows(p.n_rows, b, p.max_rows, p.status);
@@ -352,16 +363,6 @@ __global__ void __launch_bounds__(ScanCfg<N, ACC>::THREADS, N <= 16 ? SC_CTAS_PE
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);
-  }
-  // The last CTA to finish returns the tile counter to zero for the next
-  // launch (every CTA's producer has stopped taking tiles by then).
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-      p.sched[0] = 0u;
-      p.sched[1] = 0u;
-      __threadfence();
-    }
   }
 }
 

@@ -103,10 +103,15 @@ const char *csa2_status_string(csa2_status s);
 /* Thread-local text of the last error returned on this thread ("" if none). */
 const char *csa2_last_error(void);
 
-/* Bytes at the start of every workspace that hold the device status word. */
+/* Bytes at the start of every workspace: the device status word (word 0)
+ * and the Full scan's tile counter (word 16), which every scan launch
+ * returns to zero before it completes.  A workspace serves one call at a
+ * time (calls enqueued on one stream, or otherwise ordered). */
 #define CSA2_WS_HEADER 256
-/* Zero the status word of a workspace (enqueued on stream).  Call once
- * before the first use of a workspace. */
+/* Zero the header of a workspace (status word and scan counter; enqueued on
+ * stream).  Call once before the first use of a workspace, and again after
+ * a call whose csa2_sync_status reported CSA2_ERR_TIMEOUT (a scan that gave
+ * up may leave its counter non-zero). */
 csa2_status csa2_workspace_init(void *ws, size_t ws_bytes, csa2_stream_t stream);
 /* Synchronise the stream, read and clear the status word: CSA2_OK, or the
  * first device-side problem recorded since the last call. */
