@@ -255,7 +255,8 @@ __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergePa
   const int32_t* gpos = sm.gpos;
   cluster_select_topk<CPM_NT, CPM_KPT>(sm.sel, key, [gpos](int e) { return gpos[e]; }, p.top_k,
                                        p.idx + (int64_t)b * p.top_k, p.idx_count + b,
-                                       /*cluster_wide=*/false);
+                                       /*cluster_wide=*/false, nullptr, /*top_window=*/true,
+                                       /*gather_finish=*/true);
 }
 
 // ------------------------------------------------------- attention merge

@@ -88,6 +88,13 @@ __device__ __forceinline__ void st_async_v4(uint32_t dst, uint4 v, uint32_t bar)
       "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
       : "memory");
 }
+__device__ __forceinline__ void st_async_v2(uint32_t dst, uint32_t a, uint32_t b, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(
+          dst),
+      "r"(a), "r"(b), "r"(bar)
+      : "memory");
+}
 // Split cluster barrier: every thread of every CTA arrives (release), and
 // later waits (acquire).  Arrivals and waits alternate per thread.
 __device__ __forceinline__ void cluster_arrive_release() {

@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(RS_NT) rescore_select_kernel(const RescorePara
   __syncthreads();
   cluster_select_topk<RS_NT, RS_KPT>(s.sel, key, id_of, p.top_k,
                                      job.idx + (int64_t)b * job.idx_stride, job.idx_count + b,
-                                     true, p.status);
+                                     true, p.status, /*top_window=*/true, /*gather_finish=*/true);
 }
 
 // --------------------------------------------- block Top-k (pool) select

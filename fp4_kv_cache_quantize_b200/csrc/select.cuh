@@ -18,9 +18,18 @@
 //     leaves one bin's warp total per lane pair) before one shared-memory
 //     atomic per bin.  Later rounds see few keys: 64 bins, one shared atomic
 //     per key in the bracket.
+//     With top_window, when the keys span more than SEL_TOP_SPAN, the first round's 16 bins
+//     cover only the SEL_TOP_SPAN key values below the maximum (two octaves
+//     of the float values the keys encode: the k largest scores lie there
+//     unless the maximum is an outlier far above them); if fewer than k keys
+//     fall there, every one of them is above the k-th, and the next round
+//     counts the rest of the range the same way.
 //   * a round ends the search when the bin's keys are exactly the ones still
 //     wanted, or when the bin is a single key value (the lowest element
-//     indices among the keys equal to it are taken).
+//     indices among the keys equal to it are taken), or (with gather_finish)
+//     when the bin holds at most SEL_GATHER keys: then every rank sends its keys in the bin
+//     (with their element indices) to every rank, and each rank ranks the
+//     same gathered set locally, so no further counting round is needed.
 // The code runs once per CTA and every instruction of it is fetched cold
 // (instruction fetch, not arithmetic, bounds this kernel's latency), so all
 // rounds run the same rolled loop body.
@@ -47,6 +56,9 @@ namespace cg = cooperative_groups;
 
 constexpr int SEL_NB = 64;             // bins of a light round
 constexpr int SEL_MAX_RANKS = 16;
+constexpr uint32_t SEL_TOP_SPAN = 1u << 24;  // key values the first round looks at below the max
+constexpr int SEL_GATHER = 64;               // largest bin that is gathered instead of counted
+constexpr uint32_t SEL_NONE = 0xFFFFFFFFu;   // find_bin: the k-th key is below the counted range
 
 template <int NT, int KPT>
 struct SelectSmem {
@@ -60,9 +72,13 @@ struct SelectSmem {
   uint32_t verdict[4];
   uint32_t fin[4];                               // this rank's rule: T, keys == T taken, first output slot
   uint32_t wsum[32];
+  alignas(8) uint2 gbuf[SEL_GATHER];             // gathered (key, element) pairs of the final bin
+  uint32_t grank[SEL_GATHER];                    // their ranks (key descending, element ascending)
+  uint32_t gt_in[SEL_MAX_RANKS], keq[SEL_MAX_RANKS];  // per rank: gathered keys > T, taken keys == T
+  uint32_t gcnt, gT;
   uint64_t xbar[2];  // every rank's counts of the round have arrived (by parity)
   uint64_t cbar;     // every rank's round-0 figures have arrived
-  uint64_t pad_;
+  uint64_t gbar;     // the gathered bin has arrived
 };
 static_assert(sizeof(SelectSmem<256, 4>) % 16 == 0, "keeps what follows 16-byte aligned");
 
@@ -76,10 +92,16 @@ __device__ __forceinline__ void cluster_select_prologue(SelectSmem<NT, KPT>& sm,
                                                         bool cluster_wide = true) {
   const int t = threadIdx.x;
   for (int i = t; i < 2 * SEL_NB; i += NT) sm.hist[i / SEL_NB][i % SEL_NB] = 0u;
+  if (t < SEL_MAX_RANKS) {
+    sm.gt_in[t] = 0u;
+    sm.keq[t] = 0u;
+  }
   if (t == 0) {
+    sm.gcnt = 0u;
     mbar_init(&sm.xbar[0], 1);
     mbar_init(&sm.xbar[1], 1);
     mbar_init(&sm.cbar, 1);
+    mbar_init(&sm.gbar, 1);
     fence_mbar_init();
   }
   if (cluster_wide && cg::this_cluster().num_blocks() > 1) cluster_arrive_release();
@@ -166,7 +188,8 @@ __device__ __forceinline__ void count64(uint32_t* hist, const uint32_t (&key)[N]
 }
 
 // Warp 0: the bin of the krem-th largest key from per-rank counts
-// xs[r][b] (r < nr); writes (bin, keys above it, keys in it) to verdict.
+// xs[r][b] (r < nr); writes (bin, keys above it, keys in it) to verdict, or
+// (SEL_NONE, keys in the range, 0) when the range holds fewer than krem.
 template <class Smem>
 __device__ __forceinline__ void find_bin(Smem& sm, const uint32_t (*xs)[SEL_NB], unsigned nr,
                                          uint32_t krem) {
@@ -188,6 +211,12 @@ __device__ __forceinline__ void find_bin(Smem& sm, const uint32_t (*xs)[SEL_NB],
     if (lane + o < 32) suf += y;
   }
   const uint32_t above_hi = suf - pair;  // bins > 2 lane + 1
+  if (lane == 0) {  // (no bin holds it: fewer than krem keys in the range)
+    sm.verdict[0] = SEL_NONE;
+    sm.verdict[1] = suf;
+    sm.verdict[2] = 0u;
+  }
+  __syncwarp();
   if (above_hi < krem && above_hi + pair >= krem) {
     const bool in_hi = above_hi + c1 >= krem;
     sm.verdict[0] = in_hi ? 2u * lane + 1u : 2u * lane;
@@ -208,7 +237,9 @@ __device__ __forceinline__ int round_shift(uint32_t span, int bits) {
 // Writes out[0..k) (k = min(k_req, candidates)) in ascending element order,
 // out[k..k_req) = -1 and *out_count = k (rank 0 writes the last two).
 // With cluster_wide = false the calling CTA selects on its own (rank 0 of a
-// one-CTA selection) even inside a larger cluster.  A wait for another
+// one-CTA selection) even inside a larger cluster.  top_window and
+// gather_finish choose the first round's range and the last step (header
+// comment); they change the work, not the result.  A wait for another
 // rank's counts that gives up (after kWaitCycles) sets ST_TIMEOUT in
 // *status (when given) and the result is not defined.
 // cluster_select_emit: the same selection, handing each selected element to
@@ -216,7 +247,8 @@ __device__ __forceinline__ int round_shift(uint32_t span, int bits) {
 template <int NT, int KPT, class IdOf, class Emit>
 __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
                                         IdOf id_of, int k_req, Emit emit,
-                                        bool cluster_wide = true, uint32_t* status = nullptr) {
+                                        bool cluster_wide = true, uint32_t* status = nullptr,
+                                        bool top_window = false, bool gather_finish = false) {
   static_assert(NT >= 64 && NT % 32 == 0, "at least 64 threads");
   static_assert(KPT <= 15, "4-bit per-lane counters");
   static_assert(NT * KPT < 65536, "16-bit packed counts");
@@ -306,19 +338,23 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
   } else {
     uint32_t lo = gmn, hi = gmx, krem = k;
     if (t < SEL_MAX_RANKS) sm.above[t] = 0u;
-    int mode = 0;  // 1: the whole bin; 2: one key value
-    uint32_t nlo = lo, nhi = hi;
+    int mode = 0;  // 1: the whole bin; 2: one key value; 3: the bin is gathered
+    uint32_t nlo = lo, nhi = hi, inbin = 0u;
+    bool wide = true;  // this round sees every key: 16 bins in nibble counters
 #pragma unroll 1  // one copy of the body: its instructions are fetched once
-    for (int round = 0; round < 12; round++) {
-      const uint32_t span = hi - lo;  // > 0 here
+    for (int round = 0; round < 14; round++) {
       const int par = round & 1;
+      // the counted range [clo, hi]; the first round looks only below the max
+      const bool top = top_window && round == 0 && hi - lo >= SEL_TOP_SPAN;
+      const uint32_t clo = top ? hi - (SEL_TOP_SPAN - 1u) : lo;
+      const uint32_t span = hi - clo;  // > 0 here
       int s;
-      if (round == 0) {
+      if (wide) {
         s = round_shift(span, 4);
-        count16<KPT>(sm.hist[par], key, lo, span, s);
+        count16<KPT>(sm.hist[par], key, clo, span, s);
       } else {
         s = round_shift(span, 6);
-        count64<KPT>(sm.hist[par], key, lo, span, s);
+        count64<KPT>(sm.hist[par], key, clo, span, s);
       }
       __syncthreads();
       // the other parity's counts were pushed last round, before that
@@ -339,28 +375,91 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
       }
       if (wid == 0) find_bin(sm, sm.xbuf[par], ncta, krem);
       __syncthreads();
-      const uint32_t jb = sm.verdict[0], above = sm.verdict[1], inbin = sm.verdict[2];
-      for (int r = wid; r < (int)ncta; r += NW) {  // warp r: rank r's keys above the bin and in it
+      const uint32_t jb = sm.verdict[0], above = sm.verdict[1];
+      inbin = sm.verdict[2];
+      // warp r: rank r's keys above the bin (every counted key when the
+      // k-th lies below the range) and in it
+      const int jbi = jb == SEL_NONE ? -1 : (int)jb;
+      for (int r = wid; r < (int)ncta; r += NW) {
         const uint32_t* xr = sm.xbuf[par][r];
-        uint32_t a = (2 * lane > (int)jb ? xr[2 * lane] : 0u) +
-                     (2 * lane + 1 > (int)jb ? xr[2 * lane + 1] : 0u);
+        uint32_t a = (2 * lane > jbi ? xr[2 * lane] : 0u) + (2 * lane + 1 > jbi ? xr[2 * lane + 1] : 0u);
         a = __reduce_add_sync(FULL, a);
         if (lane == 0) {
           sm.above[r] += a;
-          sm.last[r] = xr[jb];
+          if (jbi >= 0) sm.last[r] = xr[jbi];
         }
       }
       krem -= above;
-      nlo = lo + (jb << s);
+      if (jb == SEL_NONE) {  // (first round only) the rest of the range, counted wide
+        hi = clo - 1u;
+        continue;
+      }
+      wide = false;
+      nlo = clo + (jb << s);
       const uint64_t h64 = (uint64_t)nlo + ((1ull << s) - 1ull);
       nhi = h64 < (uint64_t)hi ? (uint32_t)h64 : hi;
       if (inbin == krem) { mode = 1; break; }
-      if (nlo == nhi || round == 11) { mode = 2; break; }  // 32 bits take at most 6 rounds
+      if (nlo == nhi || round == 13) { mode = 2; break; }  // 32 bits take at most 7 rounds
+      if (gather_finish && inbin <= (uint32_t)SEL_GATHER) { mode = 3; break; }
       lo = nlo;
       hi = nhi;
     }
     __syncthreads();  // above / last complete
-    {
+    if (mode == 3) {
+      // ---- gather the bin: rank r's keys in [nlo, nhi] go to slots from
+      // sum_{r' < r} last[r'] on every rank; then every rank ranks them
+      uint32_t off = 0u;
+      for (unsigned r = 0; r < rank; r++) off += sm.last[r];
+      if (ncta > 1 && t == 0) mbar_arrive_expect_tx(&sm.gbar, inbin * 8u);
+      const int e0 = ((int)rank * NT + t) * KPT;
+#pragma unroll
+      for (int j = 0; j < KPT; j++) {
+        if (key[j] >= nlo && key[j] <= nhi) {
+          const uint32_t slot = off + atomicAdd(&sm.gcnt, 1u);
+          if (ncta > 1) {
+            for (unsigned r = 0; r < ncta; r++)
+              st_async_v2(mapa_rank(&sm.gbuf[slot], r), key[j], (uint32_t)(e0 + j),
+                          mapa_rank(&sm.gbar, r));
+          } else {
+            sm.gbuf[slot] = make_uint2(key[j], (uint32_t)(e0 + j));
+          }
+        }
+      }
+      if (ncta > 1) wait_counts(&sm.gbar, 0u);
+      else __syncthreads();
+      // rank of candidate i: candidates before it (key descending, element
+      // ascending); warp w takes candidates w, w + NW, ...
+      for (int i = wid; i < (int)inbin; i += NW) {
+        const uint2 ci = sm.gbuf[i];
+        uint32_t c = 0u;
+        for (int j = lane; j < (int)inbin; j += 32) {
+          const uint2 cj = sm.gbuf[j];
+          c += cj.x > ci.x || (cj.x == ci.x && cj.y < ci.y);
+        }
+        c = __reduce_add_sync(FULL, c);
+        if (lane == 0) {
+          sm.grank[i] = c;
+          if (c == krem - 1u) sm.gT = ci.x;  // the k-th largest key
+        }
+      }
+      __syncthreads();
+      const uint32_t T = sm.gT;
+      if (t < (int)inbin) {
+        const uint2 ci = sm.gbuf[t];
+        const uint32_t src = ci.y / (uint32_t)(NT * KPT);
+        if (ci.x > T) atomicAdd(&sm.gt_in[src], 1u);
+        else if (ci.x == T && sm.grank[t] < krem) atomicAdd(&sm.keq[src], 1u);
+      }
+      __syncthreads();
+      if (t == 0) {
+        uint32_t o = 0u;
+        for (unsigned r = 0; r < rank; r++) o += sm.above[r] + sm.gt_in[r] + sm.keq[r];
+        sm.fin[0] = T;
+        sm.fin[1] = sm.keq[rank];
+        sm.fin[2] = o;
+      }
+      __syncthreads();
+    } else {
       if (wid == 0) {
         // lane r = rank r.  mode 1: every key of the bin (>= nlo); mode 2:
         // the first krem keys == nlo in element order (ranks in order)
@@ -420,9 +519,11 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
 template <int NT, int KPT, class IdOf>
 __device__ void cluster_select_topk(SelectSmem<NT, KPT>& sm, const uint32_t (&key)[KPT],
                                     IdOf id_of, int k_req, int32_t* out, int32_t* out_count,
-                                    bool cluster_wide = true, uint32_t* status = nullptr) {
+                                    bool cluster_wide = true, uint32_t* status = nullptr,
+                                    bool top_window = false, bool gather_finish = false) {
   const uint32_t k = cluster_select_emit(
-      sm, key, id_of, k_req, [out](int pos, int id) { out[pos] = id; }, cluster_wide, status);
+      sm, key, id_of, k_req, [out](int pos, int id) { out[pos] = id; }, cluster_wide, status,
+      top_window, gather_finish);
   const unsigned rank = cluster_wide ? cg::this_cluster().block_rank() : 0u;
   if (rank == 0) {
     for (int i = (int)k + (int)threadIdx.x; i < k_req; i += NT) out[i] = -1;
