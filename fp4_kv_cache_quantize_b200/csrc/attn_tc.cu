@@ -47,6 +47,7 @@ constexpr int TA_TPR = TA_NT / 128;  // threads per key row (4): a quarter of th
 constexpr int TA_KEYS = 128;                        // keys per CTA: the MMA's M
 constexpr int TA_SPARSE = CSA2_MAX_TOPK / TA_KEYS;  // CTAs of the sparse branch
 constexpr int TA_CTAS = TA_SPARSE + 1;              // and the window's
+static_assert(TA_CTAS == ATTN_TC_CTAS_PER_UNIT, "cluster size the launcher plans with");
 static_assert(CSA2_W == TA_KEYS, "one CTA holds the whole window");
 constexpr int TA_KB = TA_KEYS * 128;                // one 64-channel block of the tile
 constexpr uint32_t TA_IDESC_QK = idesc_f16_f32(128, 16, false);

@@ -413,6 +413,18 @@ static csa2_status fill_attn_common(AttnParams& ap, const csa2_kv_view* kv, cons
   return CSA2_OK;
 }
 
+// Attention for every (layer, sequence) unit of a launch.  The tensor-core
+// kernel runs one 5-CTA cluster per unit at one CTA per SM: the shape for a
+// decode step whose units fit in about two waves of it.  Larger batches (many
+// sequences, or many queries per sequence) run the split-KV kernel instead,
+// several small CTAs per SM with their partials merged through L2, which
+// keeps more units in flight.
+static cudaError_t launch_attention(const AttnParams& ap, cudaStream_t st) {
+  const int64_t ctas = (int64_t)ap.batch * ap.n_layers * ATTN_TC_CTAS_PER_UNIT;
+  if (ctas > 2LL * num_sms()) return launch_attn(ap, st, /*merge=*/true);
+  return launch_attn_tc(ap, st);
+}
+
 csa2_status csa2_sparse_attn_decode(const uint16_t* q, const csa2_kv_view* kv, const int32_t* idx,
                                     const int32_t* idx_count, int32_t idx_stride,
                                     const uint8_t* swa, const int32_t* swa_len, float sm_scale,
@@ -442,7 +454,7 @@ csa2_status csa2_sparse_attn_decode(const uint16_t* q, const csa2_kv_view* kv, c
   ap.part_o = reinterpret_cast<float*>(base + CSA2_WS_HEADER);
   ap.part_ml = reinterpret_cast<float*>(base + CSA2_WS_HEADER + slots * CSA2_H * CSA2_D * 4);
   ap.status = static_cast<uint32_t*>(ws);
-  CSA2_CUDA(launch_attn_tc(ap, (cudaStream_t)stream));
+  CSA2_CUDA(launch_attention(ap, (cudaStream_t)stream));
   trace_mark("end", (cudaStream_t)stream);
   return CSA2_OK;
 }
@@ -546,7 +558,7 @@ csa2_status csa2_layer_group(const csa2_group_desc* d, void* ws, size_t ws_bytes
                             reuse ? layer_cnt(l) : nullptr,
                             d->out + (size_t)l * VB * CSA2_H * CSA2_D};
   }
-  CSA2_CUDA(launch_attn_tc(ap, st));
+  CSA2_CUDA(launch_attention(ap, st));
   trace_mark("end", st);
   return CSA2_OK;
 }

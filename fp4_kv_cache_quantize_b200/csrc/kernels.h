@@ -137,6 +137,7 @@ size_t attn_partial_bytes(int batch, int n_layers, int nsplit);
 cudaError_t launch_attn(const AttnParams& p, cudaStream_t st, bool merge = true);
 // The tensor-core attention: one 5-CTA cluster per (layer, sequence), merged
 // in the cluster, bf16 output (part_o / part_ml unused).
+constexpr int ATTN_TC_CTAS_PER_UNIT = 5;  // attn_tc_kernel: CTAs (one cluster) per (layer, sequence)
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t st);
 
 // ------------------------------------------------------------ cache append
