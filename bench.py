@@ -62,6 +62,18 @@ def measured_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def profile_value(name, key):
+    """An integer recorded as `key: value` in a committed ncu summary."""
+    try:
+        with open(os.path.join(ROOT, "profiles", name)) as fh:
+            for line in fh:
+                if line.startswith(key + ":"):
+                    return int(line.split(":", 1)[1].strip().split()[0])
+    except OSError:
+        pass
+    return None
+
+
 def scan_traffic_from_profile():
     """dram bytes per scan launch from the committed ncu summary, if any."""
     path = os.path.join(ROOT, "profiles", "scan_decoder20_1m.md")
@@ -543,7 +555,11 @@ def time_context_parallel(csa2, wl, bufs, grp, stream, flush_l2, K, W, world=8):
         graph_note = f"{type(exc).__name__}: {exc}"[:200]
     # this library's kernel launches per shard and step (the exchanges' copies excluded)
     modes, hsi = [int(m) for m in wl.modes], wl.pool_blocks > 0
-    per_shard = 1 + wl.L + 3
+    # (local rows, one filter launch for every layer, attention partial and its
+    # local merge, combine; per scan: scan, pool select, block filter, the
+    # regroup when batch > 1, and per chunk of at most CP_MAX_JOBS jobs one
+    # rescore, one export and one merge launch)
+    per_shard = 1 + 1 + 3
     for l, m in enumerate(modes):
         if m == 2 or (m == 1 and hsi):
             continue
@@ -553,7 +569,8 @@ def time_context_parallel(csa2, wl, bufs, grp, stream, flush_l2, K, W, world=8):
                 if x == 0:
                     break
                 jobs += x == 1
-        per_shard += 3 + (1 if wl.B > 1 and world > 1 else 0) + 3 * jobs
+        chunks = -(-jobs // csa2.CP_MAX_JOBS)
+        per_shard += 3 + (1 if wl.B > 1 and world > 1 else 0) + 3 * chunks
     out = {"world": world, "shard_rows": S, "ms_per_step_one_gpu_emulation": ms_direct,
            "ms_per_step_one_gpu_emulation_graph": ms_graph,
            "launches_per_shard": per_shard, "steps": K, "warmup": W,
@@ -829,7 +846,9 @@ def time_quant(csa2, dev, stream, K, W, with_cpu):
         out[name] = {"us_per_launch": t * 1e6, "value": gbs, "unit": "GB/s",
                      "roofline": {"bound": "hbm", "kernel": f"fp4_{'pack' if name == 'quantize' else 'unpack'}_kernel",
                                   "achieved": gbs, "peak": peak, "peak_kind": peak_kind,
-                                  "unit": "GB/s", "frac": gbs / peak, "traffic": None},
+                                  "unit": "GB/s", "frac": gbs / peak,
+                                  "traffic": profile_value("fp4_quant_1Mx512.md",
+                                                           f"dram_bytes_per_launch_{name}")},
                      "timing": f"{K} back-to-back launches after {W}, CUDA events (1 GiB input > L2)"}
     if with_cpu:
         import oracle
@@ -867,6 +886,15 @@ def run_gpu(args, wl, rank, world):
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
+
+    if args.quant_only:  # the FP4 quantise / dequantise leg alone (its own line)
+        stream = torch.cuda.current_stream()
+        q = time_quant(csa2, dev, stream, args.steps, args.warmup,
+                       rank == 0 and world == 1 and not args.no_cpu)
+        if rank == 0:
+            print(json.dumps({"metric": "FP4 quantise / dequantise GB/s (algorithmic bytes)",
+                              "n_gpus": world, **q}), flush=True)
+        return
 
     def to_dev(a):
         a = np.ascontiguousarray(a)
@@ -1192,6 +1220,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--skip-configs", action="store_true",
                     help="time only the headline workload (not configs 1, 2 and 4)")
+    ap.add_argument("--quant-only", action="store_true",
+                    help="time only the FP4 quantise / dequantise leg (1M x 512 rows)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", 0))

@@ -172,33 +172,36 @@ def cp_layer_group(ranks, comm, modes, n_rows, q_idx, w, q, swa, swa_len, *,
                     break
                 if modes[x] == REINDEX:
                     jobs.append(x)
-        J = len(jobs)
         for r, g in zip(ranks, bm_all):
             # the global candidate blocks (the pool, or top_k blocks without
             # one), then those this shard owns, as local block ids
             blocks, count = (r.pool, r.pool_count) if hsi else (r.blocks, r.blocks_count)
             csa2.csa2_cp_pool(r.shard, g, n_rows, P, blocks, count, r.ws)
             csa2.csa2_cp_filter(r.shard, csa2.BLK, blocks, count, r.cand, r.cand_count, r.ws)
-            for j, x in enumerate(jobs):
-                csa2.csa2_cp_select_local(r.shard, r.kv, q_idx[x], w[x], r.cand, r.cand_count, K,
-                                          r.send_sel[j], r.ws)
-        sel_all = comm.all_gather([r.send_sel[:J] for r in ranks])
-        for r, g in zip(ranks, sel_all):
-            for j, x in enumerate(jobs):
-                csa2.csa2_cp_select_merge(r.shard, g, J, j, B, K, r.idx[x], r.idx_count[x], r.ws)
+        # the jobs' local selections (one launch pair per chunk of jobs), one
+        # exchange and one merge launch per chunk
+        for c0 in range(0, len(jobs), csa2.CP_MAX_JOBS):
+            chunk = jobs[c0:c0 + csa2.CP_MAX_JOBS]
+            J = len(chunk)
+            for r in ranks:
+                csa2.csa2_cp_select_local_jobs(r.shard, r.kv, chunk, q_idx, w, r.cand,
+                                               r.cand_count, K, r.send_sel[:J], r.ws)
+            sel_all = comm.all_gather([r.send_sel[:J] for r in ranks])
+            for r, g in zip(ranks, sel_all):
+                csa2.csa2_cp_select_merge_jobs(r.shard, g, chunk, B, K, r.idx, r.idx_count, r.ws)
 
     # Attention: each shard over the selected rows it owns (+ the window on
     # window_rank), one exchange of the partials, one merge.
+    # every layer's source of indices: itself, or (REUSE) the latest FULL /
+    # REINDEX layer, whose indices it also publishes
+    src, cur = [], 0
+    for l in range(L):
+        if modes[l] != REUSE:
+            cur = l
+        src.append(cur)
     for r in ranks:
-        src = 0
-        for l in range(L):
-            reuse = modes[l] == REUSE
-            if not reuse:
-                src = l
-            csa2.csa2_cp_filter(r.shard, 1, r.idx[src], r.idx_count[src], r.idx_local[l],
-                                r.idx_local_count[l], r.ws,
-                                copy=r.idx[l] if reuse else None,
-                                copy_count=r.idx_count[l] if reuse else None)
+        csa2.csa2_cp_filter_layers(r.shard, src, r.idx, r.idx_count, r.idx_local,
+                                   r.idx_local_count, r.ws)
         win = swa_len if int(r.shard.rank) == window_rank else r.no_window
         csa2.csa2_cp_attn_partial(r.shard, r.kv, q, swa, win, r.idx_local, r.idx_local_count,
                                   sm_scale, r.partial, r.ws)

@@ -116,6 +116,14 @@ _cp_select_local = _sig("csa2_cp_select_local", C.c_int,
                          _vp])
 _cp_select_merge = _sig("csa2_cp_select_merge", C.c_int,
                         [_PS, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp])
+_cp_select_local_jobs = _sig("csa2_cp_select_local_jobs", C.c_int,
+                             [_PS, C.POINTER(KVView), _i32, _vp, _i32, _vp, _vp, _vp, _vp, _i32,
+                              _i32, _vp, _vp, _sz, _vp])
+_cp_select_merge_jobs = _sig("csa2_cp_select_merge_jobs", C.c_int,
+                             [_PS, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp])
+_cp_filter_layers = _sig("csa2_cp_filter_layers", C.c_int,
+                         [_PS, _i32, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _sz, _vp])
+CP_MAX_JOBS = 8
 _cp_attn_partial = _sig("csa2_cp_attn_partial", C.c_int,
                         [_PS, C.POINTER(KVView), _i32, _vp, _vp, _vp, _vp, _vp, _i32, C.c_float,
                          _vp, _vp, _sz, _vp])
@@ -358,6 +366,41 @@ def csa2_cp_select_merge(shard: CpShard, gathered, n_jobs, job, batch, top_k, id
     _check(_cp_select_merge(C.byref(shard), _ptr(gathered), n_jobs, job, batch, top_k,
                             _ptr(idx), _ptr(idx_count), _ptr(ws), ws.numel(),
                             _stream(stream)))
+
+
+def _host_i32(values):
+    arr = (C.c_int32 * len(values))(*[int(v) for v in values])
+    return arr
+
+
+def csa2_cp_select_local_jobs(shard: CpShard, kv: KVCache, layers, q_idx, w, cand, cand_count,
+                              top_k, send, ws, stream=None):
+    """Jobs = layers (host list) of q_idx [L][B][8][64] / w [L][B][8]; send
+    [J][B][top_k][2] (see csa2.h)."""
+    arr = _host_i32(layers)
+    _check(_cp_select_local_jobs(C.byref(shard), C.byref(kv.view), len(layers), arr,
+                                 int(q_idx.shape[0]), _ptr(q_idx), _ptr(w), _ptr(cand),
+                                 _ptr(cand_count), int(cand.shape[-1]), top_k, _ptr(send),
+                                 _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_cp_select_merge_jobs(shard: CpShard, gathered, layers, batch, top_k, idx, idx_count,
+                              ws, stream=None):
+    """Jobs 0..J-1 of gathered -> layers (host list) of idx [L][B][top_k]."""
+    arr = _host_i32(layers)
+    _check(_cp_select_merge_jobs(C.byref(shard), _ptr(gathered), len(layers), arr,
+                                 int(idx.shape[0]), batch, top_k, _ptr(idx), _ptr(idx_count),
+                                 _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_cp_filter_layers(shard: CpShard, src, idx, idx_count, idx_local, idx_local_count, ws,
+                          stream=None):
+    """Every layer's rows this shard owns: idx [L][B][K] -> idx_local (src:
+    host list of the layer each layer reads; see csa2.h)."""
+    arr = _host_i32(src)
+    _check(_cp_filter_layers(C.byref(shard), len(src), arr, _ptr(idx), _ptr(idx_count),
+                             int(idx.shape[-1]), int(idx.shape[1]), _ptr(idx_local),
+                             _ptr(idx_local_count), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def csa2_cp_attn_partial(shard: CpShard, kv: KVCache, q, swa, swa_len, idx_local, idx_count,

@@ -276,8 +276,8 @@ static int cp_nsplit(int batch, int n_layers) {
 
 struct CpWs {
   uint32_t* status;
-  int32_t* sel;        // [batch][top_k] local Top-k
-  int32_t* sel_count;  // [batch]
+  int32_t* sel;        // [jobs][batch][top_k] local Top-k
+  int32_t* sel_count;  // [jobs][batch]
   float* part_o;       // attention split partials
   float* part_ml;
   float* bm;           // [batch][world * S / 8] regrouped block maxima
@@ -289,12 +289,14 @@ static CpWs cp_ws_layout(const csa2_cp_shard* sh, int batch, int n_layers, int t
                          uint8_t* base) {
   CpWs w{};
   w.nsplit = cp_nsplit(batch, n_layers);
+  // local selections of up to RS_MAX_JOBS jobs (no more than the layers)
+  const size_t n_sel = n_layers < RS_MAX_JOBS ? (size_t)n_layers : (size_t)RS_MAX_JOBS;
   size_t off = CSA2_WS_HEADER;
   w.status = reinterpret_cast<uint32_t*>(base);
   w.sel = reinterpret_cast<int32_t*>(base + off);
-  off = align256(off + (size_t)batch * top_k * sizeof(int32_t));
+  off = align256(off + n_sel * batch * top_k * sizeof(int32_t));
   w.sel_count = reinterpret_cast<int32_t*>(base + off);
-  off = align256(off + (size_t)batch * sizeof(int32_t));
+  off = align256(off + n_sel * batch * sizeof(int32_t));
   const size_t slots = (size_t)batch * n_layers * w.nsplit;
   w.part_o = reinterpret_cast<float*>(base + off);
   w.part_ml = reinterpret_cast<float*>(base + off + slots * CSA2_H * CSA2_D * sizeof(float));
@@ -718,47 +720,112 @@ csa2_status csa2_cp_filter(const csa2_cp_shard* sh, int32_t unit, const int32_t*
   CSA2_REQUIRE(out_stride >= 1 && out_stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
                "out_stride = %d outside [1, %d]", out_stride, (int)CSA2_MAX_POOL);
   CpFilterParams p{};
-  p.list = list;
-  p.count = count;
+  p.n_lists = 1;
+  p.list[0] = list;
+  p.count[0] = count;
+  p.out[0] = out;
+  p.out_count[0] = out_count;
+  p.copy[0] = copy;
+  p.copy_count[0] = copy_count;
   p.stride = stride;
   p.lo = sh->rank * (sh->shard_rows / unit);
   p.hi = p.lo + sh->shard_rows / unit;
-  p.out = out;
-  p.out_count = out_count;
   p.out_stride = out_stride;
-  p.copy = copy;
-  p.copy_count = copy_count;
   p.status = static_cast<uint32_t*>(ws);
   CSA2_CUDA(launch_cp_filter(p, batch, (cudaStream_t)stream));
   return CSA2_OK;
 }
 
-csa2_status csa2_cp_select_local(const csa2_cp_shard* sh, const csa2_kv_view* kv,
-                                 const uint16_t* q_idx, const float* w, const int32_t* cand,
-                                 const int32_t* cand_count, int32_t cand_stride, int32_t top_k,
-                                 uint32_t* send, void* ws, size_t ws_bytes,
-                                 csa2_stream_t stream) {
+csa2_status csa2_cp_filter_layers(const csa2_cp_shard* sh, int32_t n_layers, const int32_t* src,
+                                  int32_t* idx, int32_t* idx_count, int32_t stride,
+                                  int32_t batch, int32_t* idx_local, int32_t* idx_local_count,
+                                  void* ws, size_t ws_bytes, csa2_stream_t stream) {
+  csa2_status r = check_shard(sh);
+  if (r) return r;
+  CSA2_REQUIRE(n_layers >= 1 && n_layers <= CP_MAX_LISTS, CSA2_ERR_SHAPE,
+               "n_layers = %d outside [1, %d]", n_layers, (int)CP_MAX_LISTS);
+  CSA2_REQUIRE(src != nullptr, CSA2_ERR_INVALID_ARG, "src is NULL");
+  for (int l = 0; l < n_layers; l++) {
+    CSA2_REQUIRE(src[l] >= 0 && src[l] <= l && src[src[l]] == src[l], CSA2_ERR_INVALID_ARG,
+                 "src[%d] = %d: each layer reads itself or an earlier layer that reads itself",
+                 l, src[l]);
+  }
+  CSA2_REQUIRE_I32(idx);
+  CSA2_REQUIRE_I32(idx_count);
+  CSA2_REQUIRE_I32(idx_local);
+  CSA2_REQUIRE_I32(idx_local_count);
+  CSA2_REQUIRE_PTR(ws);
+  CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
+               ws_bytes, CSA2_WS_HEADER);
+  CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
+  CSA2_REQUIRE(stride >= 1 && stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
+               "stride = %d outside [1, %d]", stride, (int)CSA2_MAX_POOL);
+  CpFilterParams p{};
+  p.n_lists = n_layers;
+  const int64_t ls = (int64_t)batch * stride;  // one layer's index list
+  for (int l = 0; l < n_layers; l++) {
+    p.list[l] = idx + src[l] * ls;
+    p.count[l] = idx_count + (int64_t)src[l] * batch;
+    p.out[l] = idx_local + l * ls;
+    p.out_count[l] = idx_local_count + (int64_t)l * batch;
+    p.copy[l] = src[l] != l ? idx + l * ls : nullptr;
+    p.copy_count[l] = src[l] != l ? idx_count + (int64_t)l * batch : nullptr;
+  }
+  p.stride = stride;
+  p.lo = sh->rank * sh->shard_rows;
+  p.hi = p.lo + sh->shard_rows;
+  p.out_stride = stride;
+  p.status = static_cast<uint32_t*>(ws);
+  CSA2_CUDA(launch_cp_filter(p, batch, (cudaStream_t)stream));
+  return CSA2_OK;
+}
+
+}  // extern "C"
+
+namespace csa2 {
+// The shard's Top-k of n_jobs jobs over one candidate list: one rescore
+// launch (a cluster per (job, sequence)) and one export launch.
+static csa2_status cp_select_local_impl(const csa2_cp_shard* sh, const csa2_kv_view* kv,
+                                        int n_jobs, const uint16_t* const* q_idx,
+                                        const float* const* w, const int32_t* cand,
+                                        const int32_t* cand_count, int32_t cand_stride,
+                                        int32_t top_k, uint2* const* send, void* ws,
+                                        size_t ws_bytes, cudaStream_t st) {
   csa2_status r = check_shard_kv(sh, kv);
   if (r) return r;
   if ((r = check_topk(top_k, 0))) return r;
-  CSA2_REQUIRE_PTR(q_idx);
-  CSA2_REQUIRE_PTR(w);
+  for (int j = 0; j < n_jobs; j++) {
+    CSA2_REQUIRE(q_idx[j] != nullptr && aligned16(q_idx[j]), CSA2_ERR_ALIGNMENT,
+                 "job %d: q_idx is NULL or not 16-byte aligned", j);
+    CSA2_REQUIRE(w[j] != nullptr && aligned16(w[j]), CSA2_ERR_ALIGNMENT,
+                 "job %d: w is NULL or not 16-byte aligned", j);
+    CSA2_REQUIRE(send[j] != nullptr && (reinterpret_cast<uintptr_t>(send[j]) & 7u) == 0,
+                 CSA2_ERR_ALIGNMENT, "send is NULL or not 8-byte aligned");
+  }
   CSA2_REQUIRE_I32(cand);
   CSA2_REQUIRE_I32(cand_count);
-  CSA2_REQUIRE(send != nullptr && (reinterpret_cast<uintptr_t>(send) & 7u) == 0,
-               CSA2_ERR_ALIGNMENT, "send is NULL or not 8-byte aligned");
   CSA2_REQUIRE_PTR(ws);
   CSA2_REQUIRE(cand_stride >= 1 && cand_stride <= CSA2_MAX_POOL, CSA2_ERR_SHAPE,
                "cand_stride = %d outside [1, %d]", cand_stride, (int)CSA2_MAX_POOL);
-  const CpWs lay = cp_ws_layout(sh, kv->batch, 1, top_k, static_cast<uint8_t*>(ws));
+  const CpWs lay = cp_ws_layout(sh, kv->batch, n_jobs, top_k, static_cast<uint8_t*>(ws));
   const size_t need = reinterpret_cast<uint8_t*>(lay.part_o) - static_cast<uint8_t*>(ws);
   CSA2_REQUIRE(ws_bytes >= need, CSA2_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
-  cudaStream_t st = (cudaStream_t)stream;
+  const int B = kv->batch;
   RescoreParams rp = rescore_params(kv, cand, cand_count, cand_stride, top_k, lay.status);
-  rp.job[0] = RescoreJob{q_idx, w, lay.sel, lay.sel_count, top_k};
-  trace_mark("rescore", st);
-  CSA2_CUDA(launch_rescore(rp, 1, kv->batch, cand_blocks_max(kv, cand_stride), st));
   CpExportParams xp{};
+  for (int j = 0; j < n_jobs; j++) {
+    int32_t* sel = lay.sel + (int64_t)j * B * top_k;
+    int32_t* sel_count = lay.sel_count + (int64_t)j * B;
+    rp.job[j] = RescoreJob{q_idx[j], w[j], sel, sel_count, top_k};
+    xp.q_idx[j] = q_idx[j];
+    xp.w[j] = w[j];
+    xp.idx[j] = sel;
+    xp.idx_count[j] = sel_count;
+    xp.send[j] = send[j];
+  }
+  trace_mark("rescore", st);
+  CSA2_CUDA(launch_rescore(rp, n_jobs, B, cand_blocks_max(kv, cand_stride), st));
+  xp.n_jobs = n_jobs;
   xp.idx_k = kv->idx_k;
   xp.page_table = kv->page_table;
   xp.max_pages = kv->max_pages;
@@ -766,48 +833,121 @@ csa2_status csa2_cp_select_local(const csa2_cp_shard* sh, const csa2_kv_view* kv
   xp.seq_stride = kv->seq_stride;
   xp.pool_rows = kv->pool_rows;
   xp.n_rows = kv->n_rows;
-  xp.q_idx = q_idx;
-  xp.w = w;
-  xp.idx = lay.sel;
-  xp.idx_count = lay.sel_count;
   xp.top_k = top_k;
   xp.pos_base = sh->rank * sh->shard_rows;
-  xp.send = reinterpret_cast<uint2*>(send);
   xp.status = lay.status;
-  CSA2_CUDA(launch_cp_export(xp, kv->batch, st));
+  CSA2_CUDA(launch_cp_export(xp, B, st));
   return CSA2_OK;
 }
 
-csa2_status csa2_cp_select_merge(const csa2_cp_shard* sh, const uint32_t* gathered,
-                                 int32_t n_jobs, int32_t job, int32_t batch, int32_t top_k,
-                                 int32_t* idx, int32_t* idx_count, void* ws, size_t ws_bytes,
-                                 csa2_stream_t stream) {
+// The global Top-k of gathered jobs job0 .. job0 + n_sel - 1 in one launch
+// (a CTA per (sequence, job)).
+static csa2_status cp_select_merge_impl(const csa2_cp_shard* sh, const uint32_t* gathered,
+                                        int n_jobs, int job0, int n_sel, int batch, int top_k,
+                                        int32_t* const* idx, int32_t* const* idx_count,
+                                        void* ws, size_t ws_bytes, cudaStream_t st) {
   csa2_status r = check_shard(sh);
   if (r) return r;
   if ((r = check_topk(top_k, 0))) return r;
   CSA2_REQUIRE(gathered != nullptr && (reinterpret_cast<uintptr_t>(gathered) & 7u) == 0,
                CSA2_ERR_ALIGNMENT, "gathered is NULL or not 8-byte aligned");
-  CSA2_REQUIRE_I32(idx);
-  CSA2_REQUIRE_I32(idx_count);
+  for (int j = 0; j < n_sel; j++) {
+    CSA2_REQUIRE_I32(idx[j]);
+    CSA2_REQUIRE_I32(idx_count[j]);
+  }
   CSA2_REQUIRE_PTR(ws);
   CSA2_REQUIRE(ws_bytes >= CSA2_WS_HEADER, CSA2_ERR_WORKSPACE, "workspace %zu < %d bytes",
                ws_bytes, CSA2_WS_HEADER);
   CSA2_REQUIRE(batch >= 1 && batch <= 65535, CSA2_ERR_SHAPE, "batch = %d", batch);
-  CSA2_REQUIRE(n_jobs >= 1 && job >= 0 && job < n_jobs, CSA2_ERR_INVALID_ARG,
-               "job = %d, n_jobs = %d", job, n_jobs);
   CSA2_REQUIRE(sh->world * top_k <= cp_merge_capacity(), CSA2_ERR_SHAPE,
                "world x top_k = %d > %d", sh->world * top_k, cp_merge_capacity());
   CpMergeParams p{};
   p.gathered = reinterpret_cast<const uint2*>(gathered);
   p.world = sh->world;
   p.n_jobs = n_jobs;
-  p.job = job;
+  p.job0 = job0;
+  p.n_sel = n_sel;
   p.batch = batch;
   p.top_k = top_k;
-  p.idx = idx;
-  p.idx_count = idx_count;
-  CSA2_CUDA(launch_cp_merge_select(p, (cudaStream_t)stream));
+  for (int j = 0; j < n_sel; j++) {
+    p.idx[j] = idx[j];
+    p.idx_count[j] = idx_count[j];
+  }
+  CSA2_CUDA(launch_cp_merge_select(p, st));
   return CSA2_OK;
+}
+}  // namespace csa2
+
+extern "C" {
+
+csa2_status csa2_cp_select_local(const csa2_cp_shard* sh, const csa2_kv_view* kv,
+                                 const uint16_t* q_idx, const float* w, const int32_t* cand,
+                                 const int32_t* cand_count, int32_t cand_stride, int32_t top_k,
+                                 uint32_t* send, void* ws, size_t ws_bytes,
+                                 csa2_stream_t stream) {
+  uint2* s0 = reinterpret_cast<uint2*>(send);
+  return cp_select_local_impl(sh, kv, 1, &q_idx, &w, cand, cand_count, cand_stride, top_k, &s0,
+                              ws, ws_bytes, (cudaStream_t)stream);
+}
+
+csa2_status csa2_cp_select_local_jobs(const csa2_cp_shard* sh, const csa2_kv_view* kv,
+                                      int32_t n_jobs, const int32_t* layer, int32_t n_layers,
+                                      const uint16_t* q_idx, const float* w,
+                                      const int32_t* cand, const int32_t* cand_count,
+                                      int32_t cand_stride, int32_t top_k, uint32_t* send,
+                                      void* ws, size_t ws_bytes, csa2_stream_t stream) {
+  if (!kv) return fail(CSA2_ERR_INVALID_ARG, "kv is NULL");
+  CSA2_REQUIRE(n_jobs >= 1 && n_jobs <= RS_MAX_JOBS, CSA2_ERR_SHAPE,
+               "n_jobs = %d outside [1, %d]", n_jobs, (int)RS_MAX_JOBS);
+  CSA2_REQUIRE(layer != nullptr, CSA2_ERR_INVALID_ARG, "layer is NULL");
+  CSA2_REQUIRE_PTR(q_idx);
+  CSA2_REQUIRE_PTR(w);
+  CSA2_REQUIRE(send != nullptr, CSA2_ERR_INVALID_ARG, "send is NULL");
+  const uint16_t* qs[RS_MAX_JOBS];
+  const float* ws_[RS_MAX_JOBS];
+  uint2* sends[RS_MAX_JOBS];
+  const int64_t B = kv->batch;
+  for (int j = 0; j < n_jobs; j++) {
+    CSA2_REQUIRE(layer[j] >= 0 && layer[j] < n_layers, CSA2_ERR_INVALID_ARG,
+                 "layer[%d] = %d outside [0, %d)", j, layer[j], n_layers);
+    qs[j] = q_idx + layer[j] * B * CSA2_HI * CSA2_DI;
+    ws_[j] = w + layer[j] * B * CSA2_HI;
+    sends[j] = reinterpret_cast<uint2*>(send) + j * B * top_k;
+  }
+  return cp_select_local_impl(sh, kv, n_jobs, qs, ws_, cand, cand_count, cand_stride, top_k,
+                              sends, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+csa2_status csa2_cp_select_merge(const csa2_cp_shard* sh, const uint32_t* gathered,
+                                 int32_t n_jobs, int32_t job, int32_t batch, int32_t top_k,
+                                 int32_t* idx, int32_t* idx_count, void* ws, size_t ws_bytes,
+                                 csa2_stream_t stream) {
+  CSA2_REQUIRE(n_jobs >= 1 && job >= 0 && job < n_jobs, CSA2_ERR_INVALID_ARG,
+               "job = %d, n_jobs = %d", job, n_jobs);
+  return cp_select_merge_impl(sh, gathered, n_jobs, job, 1, batch, top_k, &idx, &idx_count, ws,
+                              ws_bytes, (cudaStream_t)stream);
+}
+
+csa2_status csa2_cp_select_merge_jobs(const csa2_cp_shard* sh, const uint32_t* gathered,
+                                      int32_t n_jobs, const int32_t* layer, int32_t n_layers,
+                                      int32_t batch, int32_t top_k, int32_t* idx,
+                                      int32_t* idx_count, void* ws, size_t ws_bytes,
+                                      csa2_stream_t stream) {
+  CSA2_REQUIRE(n_jobs >= 1 && n_jobs <= RS_MAX_JOBS, CSA2_ERR_SHAPE,
+               "n_jobs = %d outside [1, %d]", n_jobs, (int)RS_MAX_JOBS);
+  CSA2_REQUIRE(layer != nullptr, CSA2_ERR_INVALID_ARG, "layer is NULL");
+  CSA2_REQUIRE(idx != nullptr && idx_count != nullptr, CSA2_ERR_INVALID_ARG,
+               "idx or idx_count is NULL");
+  int32_t* outs[RS_MAX_JOBS];
+  int32_t* counts[RS_MAX_JOBS];
+  for (int j = 0; j < n_jobs; j++) {
+    CSA2_REQUIRE(layer[j] >= 0 && layer[j] < n_layers, CSA2_ERR_INVALID_ARG,
+                 "layer[%d] = %d outside [0, %d)", j, layer[j], n_layers);
+    outs[j] = idx + (int64_t)layer[j] * batch * top_k;
+    counts[j] = idx_count + (int64_t)layer[j] * batch;
+  }
+  return cp_select_merge_impl(sh, gathered, n_jobs, 0, n_jobs, batch, top_k, outs, counts, ws,
+                              ws_bytes, (cudaStream_t)stream);
 }
 
 csa2_status csa2_cp_attn_partial(const csa2_cp_shard* sh, const csa2_kv_view* kv,

@@ -67,22 +67,25 @@ __global__ void cp_bm_regroup_kernel(const float* __restrict__ src, int32_t worl
 }
 
 // ------------------------------------------------------------ range filter
-// For each sequence: out = [x - lo for x in list[:count] if lo <= x < hi], in
-// list order (ascending stays ascending), -1 padded to out_stride.  copy, when
-// given, receives the list and its count verbatim.
+// For each list u and sequence: out = [x - lo for x in list[:count] if lo <= x
+// < hi], in list order (ascending stays ascending), -1 padded to out_stride.
+// copy, when given, receives the list and its count verbatim.  One CTA per
+// (sequence, list): every layer's filter is one launch.
 constexpr int CPF_NT = 256;
 
 __global__ void __launch_bounds__(CPF_NT) cp_filter_kernel(const CpFilterParams p) {
   __shared__ uint32_t wsum[32];
   pdl_launch_dependents();
   pdl_wait();
-  const int b = blockIdx.x, t = threadIdx.x;
-  int n = p.count[b];
+  const int b = blockIdx.x, u = blockIdx.y, t = threadIdx.x;
+  const int32_t* list = p.list[u];
+  int32_t* copy = p.copy[u];
+  int n = p.count[u][b];
   if (n < 0 || n > p.stride) {
     if (t == 0) set_status(p.status, ST_DEVICE_CHECK);
     n = n < 0 ? 0 : p.stride;
   }
-  const int32_t* src = p.list + (int64_t)b * p.stride;
+  const int32_t* src = list + (int64_t)b * p.stride;
   const int per = (p.stride + CPF_NT - 1) / CPF_NT;  // <= 8: stride <= CSA2_MAX_POOL
   const int i0 = t * per;
   uint32_t mine = 0u;
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(CPF_NT) cp_filter_kernel(const CpFilterParams 
   }
   uint32_t total;
   uint32_t at = block_excl_scan<CPF_NT>(mine, wsum, total);
-  int32_t* dst = p.out + (int64_t)b * p.out_stride;
+  int32_t* dst = p.out[u] + (int64_t)b * p.out_stride;
   for (int j = 0; j < per; j++) {
     const int i = i0 + j;
     if (i < n) {
@@ -105,10 +108,10 @@ __global__ void __launch_bounds__(CPF_NT) cp_filter_kernel(const CpFilterParams 
   }
   const int m = (int)total < p.out_stride ? (int)total : p.out_stride;
   for (int i = m + t; i < p.out_stride; i += CPF_NT) dst[i] = -1;
-  if (t == 0) p.out_count[b] = m;
-  if (p.copy) {
-    for (int i = t; i < p.stride; i += CPF_NT) p.copy[(int64_t)b * p.stride + i] = src[i];
-    if (t == 0) p.copy_count[b] = n;
+  if (t == 0) p.out_count[u][b] = m;
+  if (copy) {
+    for (int i = t; i < p.stride; i += CPF_NT) copy[(int64_t)b * p.stride + i] = src[i];
+    if (t == 0) p.copy_count[u][b] = n;
   }
 }
 
@@ -144,9 +147,10 @@ constexpr int CPX_ROWS = CPX_NT / 32 * 16;  // rows per CTA
 __global__ void __launch_bounds__(CPX_NT) cp_export_kernel(const CpExportParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  const int b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int b = blockIdx.y, j = blockIdx.z, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int c = lane & 3, grp = lane >> 2;
-  int n = p.idx_count[b];
+  const int32_t* idx = p.idx[j];
+  int n = p.idx_count[j][b];
   if (n < 0 || n > p.top_k) {
     if (t == 0 && blockIdx.x == 0) set_status(p.status, ST_DEVICE_CHECK);
     n = n < 0 ? 0 : p.top_k;
@@ -156,12 +160,13 @@ __global__ void __launch_bounds__(CPX_NT) cp_export_kernel(const CpExportParams 
   uint32_t bq[8];
   {
     const uint4* qp =
-        reinterpret_cast<const uint4*>(p.q_idx + ((int64_t)b * CSA2_HI + grp) * CSA2_DI + 16 * c);
+        reinterpret_cast<const uint4*>(p.q_idx[j] + ((int64_t)b * CSA2_HI + grp) * CSA2_DI + 16 * c);
     const uint4 q0 = __ldg(qp), q1 = __ldg(qp + 1);
     bq[0] = q0.x; bq[1] = q0.y; bq[2] = q0.z; bq[3] = q0.w;
     bq[4] = q1.x; bq[5] = q1.y; bq[6] = q1.z; bq[7] = q1.w;
   }
-  const float w0 = __ldg(p.w + b * CSA2_HI + 2 * c), w1 = __ldg(p.w + b * CSA2_HI + 2 * c + 1);
+  const float w0 = __ldg(p.w[j] + b * CSA2_HI + 2 * c),
+              w1 = __ldg(p.w[j] + b * CSA2_HI + 2 * c + 1);
   const int g0 = blockIdx.x * CPX_ROWS + warp * 16;  // first row of this warp's group
   uint32_t av[2][8];
   bool valid[2];
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(CPX_NT) cp_export_kernel(const CpExportParams 
 #pragma unroll
   for (int h = 0; h < 2; h++) {
     const int e = g0 + grp + 8 * h;
-    pos[h] = e < n ? p.idx[(int64_t)b * p.top_k + e] : -1;
+    pos[h] = e < n ? idx[(int64_t)b * p.top_k + e] : -1;
     valid[h] = pos[h] >= 0 && pos[h] < C;
     if (e < n && !valid[h]) set_status(p.status, ST_DEVICE_CHECK);
     int64_t row = -1;
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(CPX_NT) cp_export_kernel(const CpExportParams 
       if (e < p.top_k) {
         uint2 v = make_uint2(0u, 0xFFFFFFFFu);
         if (valid[h]) v = make_uint2(float_key(s[h]), (uint32_t)(pos[h] + p.pos_base));
-        p.send[(int64_t)b * p.top_k + e] = v;
+        p.send[j][(int64_t)b * p.top_k + e] = v;
       }
     }
   }
@@ -224,7 +229,7 @@ struct CpMergeSmem {
   int32_t gpos[CPM_NT * CPM_KPT];
 };
 
-// One CTA per sequence: element e = g * top_k + i is entry i of rank g's list;
+// One CTA per (sequence, job): element e = g * top_k + i is entry i of rank g's list;
 // rank-major order with ascending positions inside each rank is ascending
 // global position, so the selection's element-order tie rule is the
 // lower-position rule and its element-order output is ascending.
@@ -234,7 +239,8 @@ __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergePa
   pdl_launch_dependents();
   cluster_select_prologue(sm.sel, /*cluster_wide=*/false);
   pdl_wait();
-  const int b = blockIdx.x, t = threadIdx.x;
+  const int b = blockIdx.x, jl = blockIdx.y, t = threadIdx.x;
+  const int job = p.job0 + jl;
   const int n = p.world * p.top_k;  // <= CPM_NT * CPM_KPT, checked by the host
   uint32_t key[CPM_KPT];
 #pragma unroll
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergePa
     sm.gpos[e] = -1;
     if (e < n) {
       const int g = e / p.top_k, i = e - g * p.top_k;
-      const uint2 v = p.gathered[(((int64_t)g * p.n_jobs + p.job) * p.batch + b) * p.top_k + i];
+      const uint2 v = p.gathered[(((int64_t)g * p.n_jobs + job) * p.batch + b) * p.top_k + i];
       if (v.x != 0u) {
         key[j] = v.x;
         sm.gpos[e] = (int32_t)v.y;
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(CPM_NT) cp_merge_select_kernel(const CpMergePa
   __syncthreads();
   const int32_t* gpos = sm.gpos;
   cluster_select_topk<CPM_NT, CPM_KPT>(sm.sel, key, [gpos](int e) { return gpos[e]; }, p.top_k,
-                                       p.idx + (int64_t)b * p.top_k, p.idx_count + b,
+                                       p.idx[jl] + (int64_t)b * p.top_k, p.idx_count[jl] + b,
                                        /*cluster_wide=*/false, nullptr, /*top_window=*/true,
                                        /*gather_finish=*/true);
 }
@@ -367,13 +373,14 @@ cudaError_t launch_cp_bm_regroup(const float* src, int world, int batch, int nb,
 
 cudaError_t launch_cp_filter(const CpFilterParams& p, int batch, cudaStream_t st) {
   trace_mark("cp_filter", st);
-  return launch_pdl(cp_filter_kernel, dim3(batch), dim3(CPF_NT), 0, st, p);
+  return launch_pdl(cp_filter_kernel, dim3(batch, p.n_lists), dim3(CPF_NT), 0, st, p);
 }
 
 cudaError_t launch_cp_export(const CpExportParams& p, int batch, cudaStream_t st) {
   trace_mark("cp_export", st);
-  return launch_pdl(cp_export_kernel, dim3((p.top_k + CPX_ROWS - 1) / CPX_ROWS, batch),
-                    dim3(CPX_NT), 0, st, p);
+  return launch_pdl(cp_export_kernel,
+                    dim3((p.top_k + CPX_ROWS - 1) / CPX_ROWS, batch, p.n_jobs), dim3(CPX_NT), 0,
+                    st, p);
 }
 
 cudaError_t launch_cp_merge_select(const CpMergeParams& p, cudaStream_t st) {
@@ -385,8 +392,8 @@ cudaError_t launch_cp_merge_select(const CpMergeParams& p, cudaStream_t st) {
   });
   if (ea != cudaSuccess) return ea;
   trace_mark("cp_merge_select", st);
-  return launch_pdl(cp_merge_select_kernel, dim3(p.batch), dim3(CPM_NT), sizeof(CpMergeSmem), st,
-                    p);
+  return launch_pdl(cp_merge_select_kernel, dim3(p.batch, p.n_sel), dim3(CPM_NT),
+                    sizeof(CpMergeSmem), st, p);
 }
 
 cudaError_t launch_cp_attn_merge(const CpAttnMergeParams& p, int n_layers, bool final_out,

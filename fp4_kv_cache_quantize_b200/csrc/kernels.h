@@ -65,6 +65,7 @@ constexpr int CSA2_WS_SCHED_WORD = 16;
 constexpr int CSA2_SCAN_QUERIES = 8;  // queries one scan launch scores (MMA N <= 64)
 
 constexpr int RS_MAX_JOBS = 8;
+static_assert(RS_MAX_JOBS == CSA2_CP_MAX_JOBS, "jobs of one rescore launch");
 struct RescoreJob {
   const uint16_t* q_idx;
   const float* w;
@@ -164,16 +165,19 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
 
 // ------------------------------------------------- context-parallel decode
 constexpr int CP_MAX_PARTS = 16;  // shards (and attention splits) one merge combines
+constexpr int CP_MAX_LISTS = AT_MAX_LAYERS;  // lists one filter launch handles
 struct CpFilterParams {
-  const int32_t* list;   // [batch][stride] ascending ids
-  const int32_t* count;  // [batch]
+  // list u (blockIdx.y, u < n_lists):
+  const int32_t* list[CP_MAX_LISTS];   // [batch][stride] ascending ids
+  const int32_t* count[CP_MAX_LISTS];  // [batch]
+  int32_t* out[CP_MAX_LISTS];          // [batch][out_stride]
+  int32_t* out_count[CP_MAX_LISTS];    // [batch]
+  int32_t* copy[CP_MAX_LISTS];         // optional verbatim copy of list / count
+  int32_t* copy_count[CP_MAX_LISTS];
+  int32_t n_lists;
   int32_t stride;        // <= CSA2_MAX_POOL
   int32_t lo, hi;        // kept: lo <= id < hi, written as id - lo
-  int32_t* out;          // [batch][out_stride]
-  int32_t* out_count;    // [batch]
   int32_t out_stride;
-  int32_t* copy;         // optional verbatim copy of list / count
-  int32_t* copy_count;
   uint32_t* status;
 };
 struct CpExportParams {
@@ -184,20 +188,24 @@ struct CpExportParams {
   int64_t seq_stride;
   int64_t pool_rows;
   const int32_t* n_rows;     // this shard's visible rows per sequence
-  const uint16_t* q_idx;     // [batch][8][64]
-  const float* w;            // [batch][8]
-  const int32_t* idx;        // [batch][top_k] local positions, ascending
-  const int32_t* idx_count;  // [batch]
+  // job j (blockIdx.z, j < n_jobs):
+  const uint16_t* q_idx[RS_MAX_JOBS];     // [batch][8][64]
+  const float* w[RS_MAX_JOBS];            // [batch][8]
+  const int32_t* idx[RS_MAX_JOBS];        // [batch][top_k] local positions, ascending
+  const int32_t* idx_count[RS_MAX_JOBS];  // [batch]
+  uint2* send[RS_MAX_JOBS];               // [batch][top_k] (key, global position)
+  int32_t n_jobs;
   int32_t top_k;
   int32_t pos_base;          // global position of local position 0
-  uint2* send;               // [batch][top_k] (key, global position)
   uint32_t* status;
 };
 struct CpMergeParams {
   const uint2* gathered;  // [world][n_jobs][batch][top_k]
-  int32_t world, n_jobs, job, batch, top_k;
-  int32_t* idx;           // [batch][top_k]
-  int32_t* idx_count;     // [batch]
+  int32_t world, n_jobs, batch, top_k;
+  // launch job j (blockIdx.y, j < n_sel) merges gathered job job0 + j into:
+  int32_t job0, n_sel;
+  int32_t* idx[RS_MAX_JOBS];        // [batch][top_k]
+  int32_t* idx_count[RS_MAX_JOBS];  // [batch]
 };
 struct CpAttnMergeParams {
   const float* part_o;

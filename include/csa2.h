@@ -463,6 +463,47 @@ csa2_status csa2_cp_select_merge(const csa2_cp_shard *sh, const uint32_t *gather
                                  int32_t *idx, int32_t *idx_count, void *ws, size_t ws_bytes,
                                  csa2_stream_t stream);
 
+/* Batched forms (one launch, or one pair of launches, instead of one per job
+ * or per layer; results identical to the per-job calls).  Jobs that share a
+ * candidate list (a FULL layer and the REINDEX layers of its pool) are
+ * layers of the group's arrays, named by host arrays of layer numbers. */
+enum { CSA2_CP_MAX_JOBS = 8 };
+
+/* csa2_cp_select_local for n_jobs jobs (1 <= n_jobs <= CSA2_CP_MAX_JOBS):
+ * job j scores with layer layer[j] of q_idx bf16 [n_layers][batch][8][64] and
+ * w fp32 [n_layers][batch][8] (layer: host int32 [n_jobs], each in
+ * [0, n_layers)) and exports to send + j * batch * top_k * 2 (send uint32
+ * [n_jobs][batch][top_k][2], as n_jobs consecutive single-job exports).  ws
+ * as for csa2_cp_workspace_size(sh, batch, n_layers >= n_jobs, top_k). */
+csa2_status csa2_cp_select_local_jobs(const csa2_cp_shard *sh, const csa2_kv_view *kv,
+                                      int32_t n_jobs, const int32_t *layer, int32_t n_layers,
+                                      const uint16_t *q_idx, const float *w,
+                                      const int32_t *cand, const int32_t *cand_count,
+                                      int32_t cand_stride, int32_t top_k, uint32_t *send,
+                                      void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* csa2_cp_select_merge for jobs 0 .. n_jobs - 1 of gathered: job j's global
+ * Top-k goes to layer layer[j] of idx int32 [n_layers][batch][top_k] and
+ * idx_count int32 [n_layers][batch] (layer: host int32 [n_jobs], each in
+ * [0, n_layers); 1 <= n_jobs <= CSA2_CP_MAX_JOBS). */
+csa2_status csa2_cp_select_merge_jobs(const csa2_cp_shard *sh, const uint32_t *gathered,
+                                      int32_t n_jobs, const int32_t *layer, int32_t n_layers,
+                                      int32_t batch, int32_t top_k, int32_t *idx,
+                                      int32_t *idx_count, void *ws, size_t ws_bytes,
+                                      csa2_stream_t stream);
+
+/* csa2_cp_filter (unit 1) for every layer: layer l keeps the positions of
+ * idx[src[l]] (idx int32 [n_layers][batch][stride], counts idx_count
+ * [n_layers][batch]) that this shard owns, as local positions, into
+ * idx_local[l] / idx_local_count[l] (same shapes); a layer with src[l] != l
+ * (a REUSE layer) also receives idx[src[l]] and its count verbatim in idx[l]
+ * / idx_count[l].  src: host int32 [n_layers] with src[l] <= l and
+ * src[src[l]] == src[l]; 1 <= n_layers <= 32; stride in [1, CSA2_MAX_POOL]. */
+csa2_status csa2_cp_filter_layers(const csa2_cp_shard *sh, int32_t n_layers, const int32_t *src,
+                                  int32_t *idx, int32_t *idx_count, int32_t stride,
+                                  int32_t batch, int32_t *idx_local, int32_t *idx_local_count,
+                                  void *ws, size_t ws_bytes, csa2_stream_t stream);
+
 /* The shard's attention partial for every layer: over its selected rows
  * idx_local int32 [L][batch][idx_stride] (local positions from csa2_cp_filter,
  * counts idx_count [L][batch]) and the window rows swa_len[b] (zeros on ranks

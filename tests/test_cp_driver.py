@@ -136,6 +136,28 @@ class FakeLib:
             idx[b, :len(top)] = torch.from_numpy(top.astype(np.int32))
             idx_count[b] = len(top)
 
+    CP_MAX_JOBS = 8
+
+    def csa2_cp_select_local_jobs(self, sh, kv, layers, q_idx, w, cand, cand_count, top_k, send,
+                                  ws):
+        assert 1 <= len(layers) <= self.CP_MAX_JOBS
+        for j, x in enumerate(layers):  # job j: layer x's queries, export slot j
+            self.csa2_cp_select_local(sh, kv, q_idx[x], w[x], cand, cand_count, top_k, send[j],
+                                      ws)
+
+    def csa2_cp_select_merge_jobs(self, sh, gathered, layers, B, top_k, idx, idx_count, ws):
+        for j, x in enumerate(layers):  # gathered job j -> layer x
+            self.csa2_cp_select_merge(sh, gathered, len(layers), j, B, top_k, idx[x],
+                                      idx_count[x], ws)
+
+    def csa2_cp_filter_layers(self, sh, src, idx, idx_count, idx_local, idx_local_count, ws):
+        for l, s_ in enumerate(src):
+            assert s_ <= l and src[s_] == s_
+            reuse = s_ != l
+            self.csa2_cp_filter(sh, 1, idx[s_], idx_count[s_], idx_local[l], idx_local_count[l],
+                                ws, copy=idx[l] if reuse else None,
+                                copy_count=idx_count[l] if reuse else None)
+
     def csa2_cp_attn_partial(self, sh, kv, q, swa, swa_len, idx_local, idx_count, sm_scale,
                              partial, ws):
         L, B = q.shape[0], q.shape[1]
