@@ -260,7 +260,9 @@ csa2_status csa2_index_reindex(const csa2_kv_view *kv, const uint16_t *q_idx, co
  * CSA2_NOALLOC_SCRATCH_BYTES; e.g. batch x ceil(context / 8) x 4 bytes above
  * about 2 MB) is rejected with CSA2_ERR_WORKSPACE before any launch.
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * that device current), and again whenever the device's current context is
+ * a different one (after cudaDeviceReset the module loads at a new
+ * address); make that first call before any stream capture.
  * Every call shares the one array: calls whose work overlaps on the GPU
  * (two streams, two threads) race and must be serialised by the caller.
  * Device-side range checks still clamp, but their status bit stays in the
@@ -286,7 +288,9 @@ size_t csa2_attn_workspace_size(int32_t batch, int32_t n_layers);
  *                     E4M3 window swa[b][0..swa_len[b]) ]
  *   out[b][h] = softmax_j(sm_scale * q[b][h] . key_j) . values
  * one softmax over both branches (MQA: the 16 heads share each row as K and
- * V).  No keys gives zeros.  q: bf16 [batch][16][512] (|q| < 65504);
+ * V).  No keys gives zeros.  q: bf16 [batch][16][512], any finite values
+ * (each head is scaled by a power of two into fp16's range for the MMAs and
+ * the logits are scaled back exactly);
  * idx: int32 [batch][idx_stride]; swa: uint8 E4M3 [batch][128][512];
  * swa_len: int32 [batch] (<= 128); out: bf16 [batch][16][512].  Device.
  */
