@@ -95,6 +95,37 @@ def test_cp_host_validation(lib):
     assert m(ctypes.byref(sh), p, 1, 0, 1, 513, p, p, p, 256, None) == 2   # top_k > 512
 
 
+def test_cp_batched_host_validation(lib):
+    """The batched context-parallel calls check their job and layer tables on
+    the host, before any CUDA call."""
+    from fp4_kv_cache_quantize_b200 import csa2
+    lib2 = csa2._lib
+    sh = csa2.CpShard(0, 2, 128)
+    p = ctypes.c_void_p(256)
+    i32 = lambda *v: (ctypes.c_int32 * len(v))(*v)  # noqa: E731
+    fl = lib2.csa2_cp_filter_layers
+    assert fl(ctypes.byref(sh), 0, i32(0), p, p, 512, 1, p, p, p, 256, None) == 2   # no layers
+    assert fl(ctypes.byref(sh), 33, i32(*range(33)), p, p, 512, 1, p, p, p, 256, None) == 2
+    assert fl(ctypes.byref(sh), 2, None, p, p, 512, 1, p, p, p, 256, None) == 1     # no table
+    # a layer reading a later layer, and one reading a layer that reads another
+    assert fl(ctypes.byref(sh), 3, i32(0, 2, 2), p, p, 512, 1, p, p, p, 256, None) == 1
+    assert fl(ctypes.byref(sh), 3, i32(0, 0, 1), p, p, 512, 1, p, p, p, 256, None) == 1
+    assert fl(ctypes.byref(sh), 2, i32(0, 0), p, p, 4096, 1, p, p, p, 256, None) == 2  # stride
+    mj = lib2.csa2_cp_select_merge_jobs
+    assert mj(ctypes.byref(sh), p, 0, i32(0), 4, 1, 512, p, p, p, 256, None) == 2    # no jobs
+    assert mj(ctypes.byref(sh), p, 9, i32(*range(9)), 9, 1, 512, p, p, p, 256, None) == 2
+    assert mj(ctypes.byref(sh), p, 2, i32(0, 4), 4, 1, 512, p, p, p, 256, None) == 1  # layer 4
+    assert mj(ctypes.byref(sh), p, 1, None, 4, 1, 512, p, p, p, 256, None) == 1
+    assert mj(ctypes.byref(sh), p, 1, i32(0), 4, 1, 513, p, p, p, 256, None) == 2    # top_k
+    lj = lib2.csa2_cp_select_local_jobs
+    assert lj(ctypes.byref(sh), None, 1, i32(0), 4, p, p, p, p, 512, 512, p, p, 256, None) == 1
+    kv = csa2.KVView()
+    assert lj(ctypes.byref(sh), ctypes.byref(kv), 9, i32(*range(9)), 9, p, p, p, p, 512, 512, p,
+              p, 256, None) == 2
+    assert lj(ctypes.byref(sh), ctypes.byref(kv), 1, i32(5), 4, p, p, p, p, 512, 512, p, p,
+              256, None) == 1
+
+
 
 def test_noalloc_checks_arguments_before_its_scratch_size():
     """csa2_index_full_noalloc validates the view and sizes like

@@ -160,3 +160,61 @@ def test_cp_rejects_bad_shards(lib):
         lib.csa2_cp_filter(lib.CpShard(0, 2, 128), 3, n.view(1, 1), n, n.view(1, 1), n,
                            lib.workspace(256))
     assert e.value.status == 1
+
+
+def test_cp_batched_calls_equal_single_calls(lib, orc):
+    """The batched entry points (all jobs of a pool, every layer's filter in
+    one launch) give bit-identical results to the per-job / per-layer calls."""
+    wl = synth.make("cp", seed=560, B=2, n_rows=[20000, 3000],
+                    modes=[FULL, REUSE, REINDEX, REUSE, FULL, REINDEX], pool_blocks=2048,
+                    swa_len=[128, 37])
+    dw = DeviceWorkload(lib, wl, orc)
+    ranks = run_cp(lib, dw, 2, paged=False)
+    K, B, L = wl.top_k, wl.B, wl.L
+    jobs = [4, 5]  # the last pool's jobs: its candidates are in every rank's cand
+    sends_b, sends_s = [], []
+    for r in ranks:
+        sb = torch.zeros((len(jobs), B, K, 2), dtype=torch.int32, device="cuda")
+        lib.csa2_cp_select_local_jobs(r.shard, r.kv, jobs, dw.q_idx, dw.w, r.cand, r.cand_count,
+                                      K, sb, r.ws)
+        ss = torch.zeros_like(sb)
+        for j, x in enumerate(jobs):
+            lib.csa2_cp_select_local(r.shard, r.kv, dw.q_idx[x], dw.w[x], r.cand, r.cand_count,
+                                     K, ss[j], r.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(sb, ss), int(r.shard.rank)
+        sends_b.append(sb)
+        sends_s.append(ss)
+    gathered = torch.stack(sends_b)  # [world][J][B][K][2]
+    r = ranks[0]
+    idx_b = torch.full((L, B, K), -7, dtype=torch.int32, device="cuda")
+    cnt_b = torch.zeros((L, B), dtype=torch.int32, device="cuda")
+    lib.csa2_cp_select_merge_jobs(r.shard, gathered, jobs, B, K, idx_b, cnt_b, r.ws)
+    for j, x in enumerate(jobs):
+        idx_s = torch.full((B, K), -7, dtype=torch.int32, device="cuda")
+        cnt_s = torch.zeros(B, dtype=torch.int32, device="cuda")
+        lib.csa2_cp_select_merge(r.shard, gathered, len(jobs), j, B, K, idx_s, cnt_s, r.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(idx_b[x], idx_s) and torch.equal(cnt_b[x], cnt_s), x
+        assert torch.equal(idx_b[x], r.idx[x]) and torch.equal(cnt_b[x], r.idx_count[x]), x
+    src = [0, 0, 2, 2, 4, 5]  # REUSE layers 1 and 3 read (and receive) layers 0 and 2
+    for r in ranks:
+        idx_a, cnt_a = r.idx.clone(), r.idx_count.clone()
+        idx_a[[1, 3]] = -5  # the REUSE targets are rewritten by the calls
+        loc_b = torch.full_like(r.idx_local, -9)
+        lcnt_b = torch.zeros_like(r.idx_local_count)
+        lib.csa2_cp_filter_layers(r.shard, src, idx_a, cnt_a, loc_b, lcnt_b, r.ws)
+        idx_c, cnt_c = r.idx.clone(), r.idx_count.clone()
+        idx_c[[1, 3]] = -5
+        loc_s = torch.full_like(r.idx_local, -9)
+        lcnt_s = torch.zeros_like(r.idx_local_count)
+        for l, s_ in enumerate(src):
+            reuse = s_ != l
+            lib.csa2_cp_filter(r.shard, 1, idx_c[s_], cnt_c[s_], loc_s[l], lcnt_s[l], r.ws,
+                               copy=idx_c[l] if reuse else None,
+                               copy_count=cnt_c[l] if reuse else None)
+        torch.cuda.synchronize()
+        assert torch.equal(loc_b, loc_s) and torch.equal(lcnt_b, lcnt_s), int(r.shard.rank)
+        assert torch.equal(idx_a, idx_c) and torch.equal(cnt_a, cnt_c)
+        assert torch.equal(idx_a, r.idx) and torch.equal(cnt_a, r.idx_count)
+        lib.csa2_sync_status(r.ws)
