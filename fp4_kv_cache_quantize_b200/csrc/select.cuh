@@ -18,18 +18,19 @@
 //     leaves one bin's warp total per lane pair) before one shared-memory
 //     atomic per bin.  Later rounds see few keys: 64 bins, one shared atomic
 //     per key in the bracket.
-//     With top_window, when the keys span more than SEL_TOP_SPAN, the first round's 16 bins
-//     cover only the SEL_TOP_SPAN key values below the maximum (two octaves
-//     of the float values the keys encode: the k largest scores lie there
-//     unless the maximum is an outlier far above them); if fewer than k keys
-//     fall there, every one of them is above the k-th, and the next round
-//     counts the rest of the range the same way.
+//     With top_window, when the keys span more than SEL_TOP_SPAN, the first
+//     round's 16 bins cover only the SEL_TOP_SPAN key values below the
+//     maximum (two octaves of the float values the keys encode: the k
+//     largest scores lie there unless the maximum is an outlier far above
+//     them); if fewer than k keys fall there, every one of them is above the
+//     k-th, and the next round counts the rest of the range the same way.
 //   * a round ends the search when the bin's keys are exactly the ones still
 //     wanted, or when the bin is a single key value (the lowest element
 //     indices among the keys equal to it are taken), or (with gather_finish)
-//     when the bin holds at most SEL_GATHER keys: then every rank sends its keys in the bin
-//     (with their element indices) to every rank, and each rank ranks the
-//     same gathered set locally, so no further counting round is needed.
+//     when the bin holds at most SEL_GATHER keys: then every rank sends its
+//     keys in the bin (with their element indices) to every rank, and each
+//     rank ranks the same gathered set locally, so no further counting round
+//     is needed.
 // The code runs once per CTA and every instruction of it is fetched cold
 // (instruction fetch, not arithmetic, bounds this kernel's latency), so all
 // rounds run the same rolled loop body.
@@ -41,9 +42,10 @@
 // Round parities alternate two receive buffers and two mbarriers; a rank can
 // send round r + 2's counts only after it has received round r + 1's from
 // every rank, which each sent after reading its round r buffer, so a buffer
-// is never overwritten while it is read.  The placement needs no further exchange: each rank knows how many
-// selected elements precede it and how many of its keys equal to the
-// threshold it takes, and places its own with one block prefix scan.
+// is never overwritten while it is read.  The placement needs no further
+// exchange: each rank knows how many selected elements precede it and how
+// many of its keys equal to the threshold it takes, and places its own with
+// one block prefix scan.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -416,6 +418,9 @@ __device__ uint32_t cluster_select_emit(SelectSmem<NT, KPT>& sm, const uint32_t 
       for (int j = 0; j < KPT; j++) {
         if (key[j] >= nlo && key[j] <= nhi) {
           const uint32_t slot = off + atomicAdd(&sm.gcnt, 1u);
+          // (always below inbin <= SEL_GATHER; a bound only in case a failed
+          // wait left the counts inconsistent)
+          if (slot >= (uint32_t)SEL_GATHER) continue;
           if (ncta > 1) {
             for (unsigned r = 0; r < ncta; r++)
               st_async_v2(mapa_rank(&sm.gbuf[slot], r), key[j], (uint32_t)(e0 + j),
