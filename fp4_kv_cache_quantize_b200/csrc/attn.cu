@@ -474,9 +474,24 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams p) {
 
 int attn_nsplit(int pairs, int num_sms) {
   const int opts[4] = {1, 2, 5, 10};
-  for (int i = 0; i < 4; i++)
-    if ((int64_t)pairs * opts[i] >= 2LL * num_sms) return opts[i];
-  return 10;
+  const int64_t slots = 2LL * num_sms;  // CTAs resident at once: two per SM
+  if ((int64_t)pairs < slots) {         // fill the GPU once
+    for (int i = 0; i < 4; i++)
+      if ((int64_t)pairs * opts[i] >= slots) return opts[i];
+    return 10;
+  }
+  // More units than resident CTAs: the whole-unit CTAs run in waves and the
+  // last, partial wave costs a full CTA time.  Split when it shortens the
+  // waves by a clear margin (a CTA's time is its share of the keys plus a
+  // fixed ~6%; a split adds the merge, ~10% of a whole-unit CTA).
+  auto cost = [&](int ns) {
+    const int64_t waves = ((int64_t)pairs * ns + slots - 1) / slots;
+    return (double)waves * (1.0 / ns + 0.06) + (ns > 1 ? 0.1 : 0.0);
+  };
+  int best = 1;
+  for (int i = 1; i < 4; i++)
+    if (cost(opts[i]) < 0.9 * cost(best)) best = opts[i];
+  return best;
 }
 
 cudaError_t launch_attn(const AttnParams& p, cudaStream_t st, bool merge) {
