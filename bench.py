@@ -202,6 +202,16 @@ def oracle_step_time(wl):
 REFERENCE_BUDGET_S = 150.0
 
 
+def reference_counts(warmup, steps, t_step, budget_s=REFERENCE_BUDGET_S):
+    """(warm-up steps, timed steps) of the reference arm: the requested counts,
+    or as many as fit the budget at t_step seconds a step (at least one of
+    each; warm-ups take at most a tenth of the budget)."""
+    fit = max(1, int(budget_s / max(t_step, 1e-6)))
+    warm = max(1, min(warmup, max(1, fit // 10)))
+    timed = max(1, min(steps, fit - warm))
+    return warm, timed
+
+
 def run_reference(args, wl, rank):
     """The oracle as the reference arm: W warm-up and K timed full steps on one
     host core, as many of each as fit the time budget (a full 1M-context step
@@ -210,11 +220,9 @@ def run_reference(args, wl, rank):
         return
     step = oracle_step_setup(wl)
     t_first = step()                     # the first warm-up step
-    fit = max(1, int(REFERENCE_BUDGET_S / max(t_first, 1e-6)))
-    warm = min(args.warmup, max(1, fit // 10))
+    warm, timed = reference_counts(args.warmup, args.steps, t_first)
     for _ in range(warm - 1):
         step()
-    timed = max(1, min(args.steps, fit - warm))
     dts = [step() for _ in range(timed)]
     dt = sum(dts) / len(dts)
     value = wl.B * wl.L / dt

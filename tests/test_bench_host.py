@@ -126,3 +126,14 @@ def test_layer_sequential_row_issues_one_step_per_layer(monkeypatch):
         assert r["indices_equal_grouped_step"] and r["out_rel_l2_vs_grouped_step"] == 0.0
         assert r["step_launch"].startswith("direct") and r["ms_per_step"] == 0.25
         assert np.isclose(r["value"], B * L / 0.25e-3)
+
+
+def test_reference_arm_counts_fit_the_budget():
+    """The reference arm runs the requested warm-up and timed steps when they
+    fit its budget, and as many as fit otherwise (at least one of each)."""
+    import bench
+    assert bench.reference_counts(3, 20, 0.5, budget_s=150) == (3, 20)
+    w, k = bench.reference_counts(10, 200, 3.8, budget_s=150)
+    assert (w, k) == (3, 36) and (w + k) * 3.8 <= 150 + 3.8
+    assert bench.reference_counts(3, 20, 400.0, budget_s=150) == (1, 1)
+    assert bench.reference_counts(0, 0, 1.0, budget_s=150) == (1, 1)
